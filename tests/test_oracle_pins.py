@@ -1,0 +1,331 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each test names the fact it checks: a number the pages print (fixtures under
+tests/golden/), a closed form, an identity of the construction, brute force
+on tiny inputs, or finite differences. A plausible slip in the oracle (a
+dropped term, a wrong sign, a transposed operand, an off-by-one in a group
+or nibble) fails at least one of them.
+"""
+
+import json
+import math
+import os
+from statistics import NormalDist
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import bf16, brute, linear, nf4
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _w(n, k, seed=0, outliers=False):
+    return synth.weight(n, k, seed=seed, outliers=outliers).float().numpy()
+
+
+# --------------------------------------------------------------------------- bf16
+
+def test_bf16_rounding_matches_torch_cast():
+    # library routine: torch's float32 -> bfloat16 cast is round-to-nearest-even
+    g = torch.Generator().manual_seed(11)
+    v = torch.randn(200000, generator=g) * torch.exp(torch.randn(200000, generator=g) * 8)
+    ours = bf16.round_to_bf16(v.numpy())
+    ref = v.to(torch.bfloat16).float().numpy()
+    assert np.array_equal(ours.view(np.uint32), ref.view(np.uint32))
+
+
+# --------------------------------------------------------------------------- codebook
+
+def test_codebook_shape_endpoints_zero():
+    c = nf4.codebook()
+    assert c.dtype == np.float32 and c.shape == (16,)
+    assert c[0] == -1.0 and c[15] == 1.0          # normalised to [-1, 1]
+    assert c[7] == 0.0                            # the exact zero
+    assert np.all(np.diff(c.astype(np.float64)) > 0)
+    assert int(np.sum(c < 0)) == 7 and int(np.sum(c > 0)) == 8
+
+
+def test_codebook_levels_are_normal_quantiles():
+    # Each level times Phi^-1(delta) must sit at its quantile point; checked with
+    # math.erf, not with the inverse CDF the oracle uses.
+    c = nf4.codebook_f64()
+    delta = 0.5 * ((1 - 1 / 30) + (1 - 1 / 32))
+    z = NormalDist().inv_cdf(delta)
+    assert abs(nf4.normal_cdf(z) - delta) < 1e-13
+    pos = sorted(delta + j * (0.5 - delta) / 8 for j in range(8))
+    neg = sorted(delta + j * (0.5 - delta) / 7 for j in range(7))
+    for i, p in enumerate(pos):           # c[8..15] ascending <-> p ascending
+        assert abs(nf4.normal_cdf(c[8 + i] * z) - p) < 1e-12
+    for i, p in enumerate(neg):           # c[6], c[5], ... c[0]: more negative as p grows
+        assert abs(nf4.normal_cdf(-c[6 - i] * z) - p) < 1e-12
+
+
+def test_codebook_dense_near_zero():
+    # levels are denser near zero than at the tails (normal quantiles)
+    gaps = np.diff(nf4.codebook_f64())
+    assert gaps[7] < gaps[14] and gaps[6] < gaps[0]
+    assert np.all(np.diff(gaps[7:]) > 0)     # positive side: gaps grow outward
+    assert np.all(np.diff(gaps[:7]) < 0)     # negative side: gaps shrink toward 0
+
+
+def test_midpoints_between_levels():
+    c = nf4.codebook().astype(np.float64)
+    m = nf4.midpoints().astype(np.float64)
+    assert m.shape == (15,)
+    assert np.all(c[:-1] < m) and np.all(m < c[1:])
+    assert np.all(np.abs(m - (c[:-1] + c[1:]) / 2) <= np.spacing(np.float32(1.0)))
+
+
+# --------------------------------------------------------------------------- storage budget
+
+def test_bit_budget_matches_pages():
+    g = _golden("bit_budget.json")
+    n, k = 8192, 22016
+    assert nf4.bits_per_param(n, k, dq=False) == g["bits_nf4_fp32_block_scale"]
+    b = nf4.bits_per_param(n, k, dq=True)
+    assert round(b, g["bits_nf4_double_quant_decimals"]) == g["bits_nf4_double_quant"]
+    # closed form 4 + 8/64 + 32/(64*256) for whole groups
+    assert b == pytest.approx(4 + 8 / 64 + 32 / (64 * 256), abs=1e-12)
+    saving_gb = (4.5 - b) / 8 * g["params_65b"] / 1e9
+    assert abs(saving_gb - g["dq_saving_65b_gb_approx"]) < g["dq_saving_65b_gb_tolerance"]
+
+
+def test_lora_param_count_matches_pages():
+    g = _golden("lora_param_count.json")
+    d, r = g["d"], g["r"]
+    a = synth.lora_a(r, d)
+    b = synth.lora_b(d, r)
+    assert a.numel() + b.numel() == g["low_rank_numbers"]
+    assert round(d * d / 1e6, 1) == g["full_numbers_millions_approx"]
+
+
+# --------------------------------------------------------------------------- quantizer
+
+@pytest.mark.parametrize("seed,outliers", [(0, False), (1, True), (2, False)])
+def test_quantizer_matches_brute_force(seed, outliers):
+    n, k = 6, 192                       # 18 blocks -> one partial DQ group
+    w = _w(n, k, seed, outliers)
+    w[2, 64:128] = 0.0                  # a zero block
+    w[4, :64] = -w[4, :64]
+    out = nf4.quantize(w)
+    levels = [float(v) for v in nf4.codebook()]
+    q_rows, scales = brute.quantize_rows(w.tolist(), levels)
+    q_b = np.array(q_rows, dtype=np.uint8)
+    # literal argmin agrees except for x within 1 ulp of a true midpoint
+    c64 = nf4.codebook_f64()
+    true_mid = (c64[:-1] + c64[1:]) / 2
+    s = np.repeat(out["absmax"], 64).reshape(n, k)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        x = np.where(s > 0, w / np.where(s > 0, s, 1), 0).astype(np.float32)
+    near = np.any(np.abs(x[..., None].astype(np.float64) - true_mid) <= 2 * np.spacing(np.float32(1.0)), axis=-1)
+    assert np.array_equal(out["q"][~near], q_b[~near])
+    assert np.array_equal(np.array(scales, dtype=np.float32), out["absmax"])
+    packed_b = np.array([brute.pack_row(r) for r in q_rows], dtype=np.uint8)
+    packed_o = nf4.pack(q_b)
+    assert np.array_equal(packed_b, packed_o)
+    q2_b, smax_b = brute.double_quantize(scales)
+    assert np.array_equal(np.array(q2_b, dtype=np.uint8), out["q2"])
+    assert np.array_equal(np.array(smax_b, dtype=np.float32), out["smax"])
+
+
+def test_zero_block_and_zero_group():
+    w = np.zeros((2, 128), dtype=np.float32)
+    out = nf4.quantize(w)
+    assert np.all(out["q"] == nf4.ZERO_CODE)
+    assert np.all(out["codes"] == 0x77)
+    assert np.all(out["q2"] == 0) and np.all(out["smax"] == 0)
+    assert np.all(nf4.dequantize(out["codes"], out["q2"], out["smax"]) == 0)
+
+
+def test_round_trip_of_levels():
+    # w = c_j * s (bf16) in a block whose max is s  ->  index j exactly
+    c = nf4.codebook()
+    s = np.float32(0.0371)
+    levels = bf16.round_to_bf16((c * s).astype(np.float32))
+    row = np.tile(levels, 4)[None, :]             # 64 values, contains +-s
+    s_b = bf16.round_to_bf16(np.array([s], np.float32))[0]
+    row[0, 15] = s_b
+    row[0, 0] = -s_b
+    q = nf4.quantize(row)["q"][0]
+    assert np.array_equal(q, np.tile(np.arange(16, dtype=np.uint8), 4))
+
+
+def test_encode_error_within_half_gap():
+    w = _w(64, 512, seed=3, outliers=True)
+    out = nf4.quantize(w)
+    s = np.repeat(out["absmax"], 64).reshape(w.shape)
+    x = (w / s).astype(np.float32).astype(np.float64)
+    c = nf4.codebook().astype(np.float64)
+    err = np.abs(x - c[out["q"]])
+    assert err.max() <= nf4.max_level_gap() / 2 + 1e-7
+
+
+def test_pack_unpack_round_trip_and_nibble_order():
+    g = np.random.default_rng(0)
+    q = g.integers(0, 16, size=(5, 64), dtype=np.uint8)
+    assert np.array_equal(nf4.unpack(nf4.pack(q)), q)
+    one = np.zeros((1, 64), dtype=np.uint8)
+    one[0, 0], one[0, 1] = 0xA, 0x3
+    assert nf4.pack(one)[0, 0] == 0xA3       # element 0 -> high nibble
+
+
+def test_outlier_touches_only_its_block_and_group():
+    w = _w(8, 4096, seed=4)                  # 512 blocks -> 2 groups of 256
+    base = nf4.quantize(w)
+    w2 = w.copy()
+    w2[3, 1000] = np.float32(bf16.round_to_bf16(np.array([w[3, 1000] * 20 + 0.5], np.float32))[0])
+    pert = nf4.quantize(w2)
+    blk = (3 * 4096 + 1000) // 64
+    grp = blk // 256
+    q_diff = np.nonzero(np.any(base["q"].reshape(-1, 64) != pert["q"].reshape(-1, 64), axis=1))[0]
+    assert set(q_diff.tolist()) <= {blk}
+    q2_diff = np.nonzero(base["q2"] != pert["q2"])[0]
+    assert set((q2_diff // 256).tolist()) <= {grp}
+    sm_diff = np.nonzero(base["smax"] != pert["smax"])[0]
+    assert set(sm_diff.tolist()) <= {grp}
+
+
+# --------------------------------------------------------------------------- double quantization
+
+def test_double_quant_error_bound():
+    w = _w(256, 4096, seed=5, outliers=True)
+    out = nf4.quantize(w)
+    s = out["absmax"].astype(np.float64)
+    s_hat = nf4.restored_scale(out["q2"], out["smax"]).astype(np.float64)
+    smax = out["smax"].astype(np.float64)[np.arange(s.size) // 256]
+    err = np.abs(s - s_hat)
+    assert np.all(err <= smax / 256 * (1 + 1e-6))              # the printed bound
+    top = out["q2"] == 255
+    assert np.all(err[~top] <= smax[~top] / 512 * (1 + 1e-6))  # every other code: half a step
+    # each group's largest block lands on the top code, restored to 255/256 of s_max
+    for g in range(out["smax"].size):
+        sl = slice(256 * g, 256 * (g + 1))
+        i = np.argmax(s[sl])
+        assert out["q2"][sl][i] == 255
+    assert nf4.n_groups(out["absmax"].size) == out["smax"].size
+
+
+def test_double_quant_extra_error_is_tiny():
+    # extra error from re-quantizing the scales stays below 0.01 % of the
+    # weight norm (relative Frobenius error, DQ minus plain fp32 scales)
+    w = _w(512, 4096, seed=6)
+    out = nf4.quantize(w)
+    c = nf4.codebook()
+    plain = (c[out["q"]].reshape(-1, 64) * out["absmax"].reshape(-1, 1)).reshape(w.shape)
+    dq = nf4.dequantize(out["codes"], out["q2"], out["smax"])
+    e_plain = linear.rel_fro(plain, w)
+    e_dq = linear.rel_fro(dq, w)
+    assert e_dq - e_plain < 1e-4
+    assert 0.0 < e_plain < 0.2
+
+
+def test_dequant_error_bound():
+    w = _w(128, 2048, seed=7, outliers=True)
+    out = nf4.quantize(w)
+    w_hat = nf4.dequantize(out["codes"], out["q2"], out["smax"]).astype(np.float64)
+    s = np.repeat(out["absmax"], 64).reshape(w.shape).astype(np.float64)
+    smax = np.repeat(out["smax"].astype(np.float64)[np.arange(out["absmax"].size) // 256], 64).reshape(w.shape)
+    bound = s * nf4.max_level_gap() / 2 + smax / 256 + np.abs(w_hat) * 2.0 ** -8
+    assert np.all(np.abs(w.astype(np.float64) - w_hat) <= bound * (1 + 1e-6))
+
+
+def test_dequant_is_bf16_of_level_times_scale():
+    # closed form per element, written with Python floats and struct-free rounding
+    w = _w(4, 256, seed=8)
+    out = nf4.quantize(w)
+    got = nf4.dequantize(out["codes"], out["q2"], out["smax"])
+    c = [float(v) for v in nf4.codebook()]
+    for n in range(4):
+        for k in range(0, 256, 7):
+            b = (n * 256 + k) // 64
+            s_hat = brute.f32_round(float(out["q2"][b]) * float(out["smax"][b // 256])) / 256.0
+            v = brute.f32_round(c[out["q"][n, k]] * s_hat)
+            ref = float(bf16.round_to_bf16(np.array([v], np.float32))[0])
+            assert got[n, k] == ref
+
+
+# --------------------------------------------------------------------------- linear
+
+def _small(m=3, n=5, k=64, r=4, seed=9):
+    g = np.random.default_rng(seed)
+    rb = lambda *s: bf16.round_to_bf16(g.standard_normal(s).astype(np.float32))
+    return rb(m, k), rb(n, k), rb(r, k), rb(n, r), rb(m, n)
+
+
+def test_forward_matches_brute_loops():
+    x, w, a, b, _ = _small()
+    s = 16.0 / 4
+    y, u = linear.forward(x, w, a, b, s)
+    yb = np.array(brute.forward(x.tolist(), w.tolist(), a.tolist(), b.tolist(), s))
+    assert np.allclose(y, yb, rtol=1e-12, atol=1e-12)
+    assert np.allclose(u, np.array(brute.matmul_nt(x.tolist(), a.tolist())), rtol=1e-12, atol=1e-12)
+
+
+def test_forward_b_zero_is_base_model():
+    x, w, a, b, _ = _small()
+    y, _ = linear.forward(x, w, a, np.zeros_like(b), 2.0)
+    assert np.array_equal(y, x.astype(np.float64) @ w.astype(np.float64).T)
+
+
+def test_forward_w_zero_is_lora_only():
+    x, w, a, b, _ = _small()
+    y, _ = linear.forward(x, np.zeros_like(w), a, b, 0.5)
+    ref = 0.5 * np.array(brute.matmul_nt(np.array(brute.matmul_nt(x.tolist(), a.tolist())).tolist(), b.tolist()))
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_backward_matches_finite_differences():
+    # L = <dY, y> is linear in each of x, A, B separately, so central
+    # differences are exact up to rounding (Proposition 1: the gradients of
+    # the LoRA path are the true gradients; W gets none).
+    p = synth.TINY
+    t = synth.make(p, seed=0)
+    w = nf4.dequantize(**{k: v for k, v in nf4.quantize(t["w"].float().numpy()).items() if k in ("codes", "q2", "smax")})
+    x, a, b, dy = (t[k].float().numpy().astype(np.float64) for k in ("x", "a", "b", "dy"))
+    x, a, b, dy = x[:4, :128], a[:, :128], b[:64], dy[:4, :64]
+    w = w[:64, :128].astype(np.float64)
+    s = p.scale
+    dx, da, db = linear.backward(x, dy, w, a, b, s)
+    h = 1e-3
+    g = np.random.default_rng(1)
+
+    def fd(arr, idx):
+        plus, minus = arr.copy(), arr.copy()
+        plus[idx] += h
+        minus[idx] -= h
+        return plus, minus
+
+    for name, arr, grad in (("x", x, dx), ("a", a, da), ("b", b, db)):
+        for _ in range(12):
+            idx = tuple(int(g.integers(0, d)) for d in arr.shape)
+            p_, m_ = fd(arr, idx)
+            args = {"x": x, "a": a, "b": b}
+            args_p = dict(args, **{name: p_})
+            args_m = dict(args, **{name: m_})
+            lp = linear.loss(args_p["x"], dy, w, args_p["a"], args_p["b"], s)
+            lm = linear.loss(args_m["x"], dy, w, args_m["a"], args_m["b"], s)
+            num = (lp - lm) / (2 * h)
+            assert abs(num - grad[idx]) <= 1e-6 * max(1.0, abs(grad[idx])), (name, idx)
+
+
+def test_backward_has_no_weight_gradient_and_b_zero():
+    # B = 0 at the start: dA vanishes, dB does not (B receives gradient in step one)
+    x, w, a, b, dy = _small()
+    dx, da, db = linear.backward(x, dy, w, a, np.zeros_like(b), 4.0)
+    assert np.all(da == 0)
+    assert np.any(db != 0)
+    assert np.array_equal(dx, dy.astype(np.float64) @ w.astype(np.float64))
+    assert len(linear.backward(x, dy, w, a, b, 4.0)) == 3     # dX, dA, dB only
+
+
+def test_rel_fro():
+    a = np.array([3.0, 4.0])
+    assert linear.rel_fro(a * 1.01, a) == pytest.approx(0.01)
