@@ -1,0 +1,648 @@
+// Host side of the C ABI (include/qlora.h): argument checks, the NF4 table,
+// workspace planning, TMA descriptors and kernel launches. No allocation,
+// no synchronisation (except qlora_device_status), no exceptions across the
+// ABI.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "../../include/qlora.h"
+#include "kernels.h"
+
+namespace qlora {
+namespace {
+
+constexpr int kBlock = 64;
+constexpr int kGroup = 256;
+constexpr int kMaxRank = 256;
+constexpr int kGemvMaxM = 16;
+
+// ------------------------------------------------------------------ NF4 table
+double normal_cdf(double z) { return 0.5 * std::erfc(-z / std::sqrt(2.0)); }
+
+// Phi^-1(p) for p in [1/2, 1) by Newton's method from z = 0. Phi is concave
+// on z >= 0, so the iterates increase monotonically to the root.
+double normal_quantile_upper(double p) {
+  const double inv_sqrt_2pi = 0.39894228040143267794;
+  double z = 0.0;
+  for (int it = 0; it < 200; ++it) {
+    const double f = normal_cdf(z) - p;
+    const double d = inv_sqrt_2pi * std::exp(-0.5 * z * z);
+    const double step = f / d;
+    z -= step;
+    if (std::fabs(step) <= 1e-17 * std::fmax(1.0, std::fabs(z))) break;
+  }
+  return z;
+}
+
+struct Tables {
+  float cb[16];
+  float mid[16];
+};
+
+const Tables& tables() {
+  static Tables t = [] {
+    Tables r{};
+    const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
+    double lv[16];
+    int n = 0;
+    for (int j = 0; j < 7; ++j) lv[n++] = -normal_quantile_upper(delta + j * (0.5 - delta) / 7.0);
+    lv[n++] = 0.0;
+    for (int j = 0; j < 8; ++j) lv[n++] = normal_quantile_upper(delta + j * (0.5 - delta) / 8.0);
+    // ascending order: the negatives grow toward 0 as j grows, the positives shrink
+    double sorted[16];
+    for (int i = 0; i < 7; ++i) sorted[i] = lv[i];          // j = 0..6: -1.x ... -0.1
+    sorted[7] = 0.0;
+    for (int i = 0; i < 8; ++i) sorted[8 + i] = lv[15 - i];  // j = 7..0
+    const double top = normal_quantile_upper(delta);
+    for (int i = 0; i < 16; ++i) r.cb[i] = static_cast<float>(sorted[i] / top);
+    for (int i = 0; i < 15; ++i)
+      r.mid[i] = static_cast<float>((static_cast<double>(r.cb[i]) + static_cast<double>(r.cb[i + 1])) / 2.0);
+    r.mid[15] = 2.0f;
+    return r;
+  }();
+  return t;
+}
+
+// ------------------------------------------------------------------ device state
+struct DevState {
+  bool checked = false;
+  bool ok = false;
+  int sms = 148;
+  bool attrs = false;
+};
+std::mutex g_mu;
+DevState g_dev[64];
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+template <int BN, int AS, int BS, int EP>
+cudaError_t set_tc_attr() {
+  return cudaFuncSetAttribute(k_tc_gemm<BN, AS, BS, EP, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              tc_smem_bytes<BN, AS, BS, 4>());
+}
+
+template <int BN>
+cudaError_t set_small_attrs() {
+  cudaError_t e;
+  if ((e = set_tc_attr<BN, A_TMA_K, B_TMA_K, EPI_F32_ROWS>()) != cudaSuccess) return e;
+  if ((e = set_tc_attr<BN, A_TMA_K, B_TMA_MN, EPI_F32_ROWS>()) != cudaSuccess) return e;
+  return set_tc_attr<BN, A_TMA_MN, B_TMA_MN, EPI_F32_ROWS>();
+}
+
+qlora_status_t device_ready(int* sms_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevState& st = g_dev[dev];
+  if (!st.checked) {
+    st.checked = true;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return QLORA_ERR_CUDA;
+    st.ok = (prop.major == 10 && prop.minor == 0);
+    st.sms = prop.multiProcessorCount;
+  }
+  if (!st.ok) return QLORA_ERR_UNSUPPORTED_DEVICE;
+  if (!st.attrs) {
+    cudaError_t e = set_tc_attr<256, A_DQ_K, B_TMA_K, EPI_BF16_T>();
+    if (e == cudaSuccess) e = set_tc_attr<256, A_DQ_MN, B_TMA_K, EPI_BF16_T>();
+    if (e == cudaSuccess) e = set_small_attrs<64>();
+    if (e == cudaSuccess) e = set_small_attrs<128>();
+    if (e == cudaSuccess) e = set_small_attrs<192>();
+    if (e == cudaSuccess) e = set_small_attrs<256>();
+    if (e != cudaSuccess) return QLORA_ERR_CUDA;
+    st.attrs = true;
+  }
+  if (sms_out) *sms_out = st.sms;
+  return QLORA_OK;
+}
+
+// ------------------------------------------------------------------ helpers
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t rup(int64_t a, int64_t b) { return cdiv(a, b) * b; }
+inline int32_t r64_of(int32_t r) { return static_cast<int32_t>(rup(r, 64)); }
+inline size_t al256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+bool map2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
+           uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// bf16 [outer x inner] row-major, 128-byte swizzled boxes of {64, box_outer}
+bool map_bf16(CUtensorMap* m, const void* ptr, int64_t outer, int64_t inner, int64_t ld, uint32_t box_outer) {
+  return map2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, inner, outer, ld * 2, 64, box_outer,
+               CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Split count for a reduction of `ktiles` 64-wide tiles over `tiles` output tiles.
+int pick_splits(int64_t tiles, int64_t ktiles, int sms) {
+  int64_t s = cdiv(sms, std::max<int64_t>(1, tiles));
+  s = std::min<int64_t>(s, ktiles);
+  s = std::min<int64_t>(s, 16);
+  s = std::max<int64_t>(s, 1);
+  const int64_t per = cdiv(ktiles, s);
+  return static_cast<int>(cdiv(ktiles, per));
+}
+
+struct SmallPlan {
+  int splits, kt_split;
+  int64_t rows_pad;
+  size_t part_bytes;
+};
+
+SmallPlan plan_small(int64_t rows, int64_t ktiles, int32_t r64, int sms) {
+  SmallPlan p;
+  const int64_t tiles = cdiv(rows, 128);
+  p.splits = pick_splits(tiles, ktiles, sms);
+  p.kt_split = static_cast<int>(cdiv(ktiles, p.splits));
+  p.rows_pad = tiles * 128;
+  p.part_bytes = static_cast<size_t>(p.splits) * p.rows_pad * r64 * sizeof(float);
+  return p;
+}
+
+struct WsPlan {
+  size_t u_pad, v_pad, b_pad, part, total;
+};
+
+WsPlan plan_ws(int64_t m, int64_t n, int64_t k, int32_t r, int sms) {
+  const int32_t r64 = r64_of(r);
+  WsPlan w{};
+  w.u_pad = al256(static_cast<size_t>(m) * r64 * 2);
+  w.v_pad = al256(static_cast<size_t>(m) * r64 * 2);
+  w.b_pad = (r % 8 != 0) ? al256(static_cast<size_t>(n) * r64 * 2) : 0;
+  size_t part = 0;
+  part = std::max(part, plan_small(m, cdiv(k, 64), r64, sms).part_bytes);   // x A^T
+  part = std::max(part, plan_small(m, cdiv(n, 64), r64, sms).part_bytes);   // dY B
+  part = std::max(part, plan_small(k, cdiv(m, 64), r64, sms).part_bytes);   // dA
+  part = std::max(part, plan_small(n, cdiv(m, 64), r64, sms).part_bytes);   // dB
+  w.part = al256(part);
+  w.total = w.u_pad + w.v_pad + w.b_pad + w.part + 256;
+  return w;
+}
+
+qlora_status_t check_nf4(const qlora_nf4_t* q) {
+  if (q == nullptr || q->codes == nullptr || q->scale_codes == nullptr || q->absmax == nullptr)
+    return QLORA_ERR_INVALID_ARG;
+  if (q->block != kBlock || q->dq_group != kGroup) return QLORA_ERR_INVALID_ARG;
+  if (q->n_out <= 0 || q->k_in <= 0 || q->k_in % kBlock != 0) return QLORA_ERR_SHAPE;
+  if (q->n_out > (int64_t(1) << 31) - 1 || q->k_in > (int64_t(1) << 31) - 1) return QLORA_ERR_SHAPE;
+  if (!aligned16(q->codes)) return QLORA_ERR_ALIGNMENT;
+  return QLORA_OK;
+}
+
+inline qlora_status_t launch_status() {
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+CUtensorMap zero_map() {
+  CUtensorMap m;
+  std::memset(&m, 0, sizeof(m));
+  return m;
+}
+
+template <int BN, int AS, int BS, int EP>
+qlora_status_t launch_tc(dim3 grid, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& b,
+                         const CUtensorMap& bl, const CUtensorMap& c, const TcParams& p) {
+  k_tc_gemm<BN, AS, BS, EP, 4><<<grid, 192, tc_smem_bytes<BN, AS, BS, 4>(), st>>>(a, b, bl, c, p);
+  return launch_status();
+}
+
+template <int AS, int BS>
+qlora_status_t launch_small(int32_t r64, dim3 grid, cudaStream_t st, const CUtensorMap& a,
+                            const CUtensorMap& b, const TcParams& p) {
+  const CUtensorMap z = zero_map();
+  switch (r64) {
+    case 64: return launch_tc<64, AS, BS, EPI_F32_ROWS>(grid, st, a, b, z, z, p);
+    case 128: return launch_tc<128, AS, BS, EPI_F32_ROWS>(grid, st, a, b, z, z, p);
+    case 192: return launch_tc<192, AS, BS, EPI_F32_ROWS>(grid, st, a, b, z, z, p);
+    case 256: return launch_tc<256, AS, BS, EPI_F32_ROWS>(grid, st, a, b, z, z, p);
+    default: return QLORA_ERR_SHAPE;
+  }
+}
+
+qlora_status_t launch_reduce(const ReduceParams& rp, int sms, cudaStream_t st) {
+  const int64_t total = static_cast<int64_t>(rp.rows) * (rp.mode == 0 ? rp.ld : rp.cols);
+  const int blocks = static_cast<int>(std::min<int64_t>(cdiv(total, 256), int64_t(sms) * 8));
+  k_reduce_splits<<<std::max(blocks, 1), 256, 0, st>>>(rp);
+  return launch_status();
+}
+
+// out_pad[rows x r64] = bf16(scale * (A_rows . B)) for a TMA-fed LoRA product
+// with the reduction over `kdim` (split over the grid's z).
+template <int AS, int BS>
+qlora_status_t lora_product(const CUtensorMap& ma, const CUtensorMap& mb, int64_t rows, int64_t kdim,
+                            int32_t r, float scale, int reduce_mode, __nv_bfloat16* out_pad,
+                            __nv_bfloat16* out_c, float* out_f, float* part, int sms,
+                            cudaStream_t st) {
+  const int32_t r64 = r64_of(r);
+  const SmallPlan sp = plan_small(rows, cdiv(kdim, 64), r64, sms);
+  TcParams p{};
+  p.rows = static_cast<int32_t>(rows);
+  p.cols = r64;
+  p.kt_main = static_cast<int32_t>(cdiv(kdim, 64));
+  p.kt_lora = 0;
+  p.kt_split = sp.kt_split;
+  p.out = part;
+  p.ldo = r64;
+  p.rows_pad = static_cast<int32_t>(sp.rows_pad);
+  const dim3 grid(static_cast<unsigned>(cdiv(rows, 128)), 1, static_cast<unsigned>(sp.splits));
+  qlora_status_t s = launch_small<AS, BS>(r64, grid, st, ma, mb, p);
+  if (s != QLORA_OK) return s;
+  ReduceParams rp{};
+  rp.part = part;
+  rp.splits = sp.splits;
+  rp.rows = static_cast<int32_t>(rows);
+  rp.rows_pad = static_cast<int32_t>(sp.rows_pad);
+  rp.ld = r64;
+  rp.cols = r;
+  rp.scale = scale;
+  rp.out_pad = out_pad;
+  rp.out_c = out_c;
+  rp.out_f = out_f;
+  rp.mode = reduce_mode;
+  return launch_reduce(rp, sms, st);
+}
+
+struct LinearArgs {
+  const qlora_nf4_t* q;
+  int64_t m;
+  int32_t r;
+  float alpha;
+  void* ws;
+  size_t ws_bytes;
+};
+
+qlora_status_t check_linear(const LinearArgs& a, int sms) {
+  qlora_status_t s = check_nf4(a.q);
+  if (s != QLORA_OK) return s;
+  if (a.m < 0 || a.m > (int64_t(1) << 31) - 1) return QLORA_ERR_SHAPE;
+  if (a.r < 1 || a.r > kMaxRank) return QLORA_ERR_SHAPE;
+  if (!std::isfinite(a.alpha)) return QLORA_ERR_INVALID_ARG;
+  if (a.m == 0) return QLORA_OK;
+  if (a.ws == nullptr || !aligned16(a.ws)) return a.ws == nullptr ? QLORA_ERR_WORKSPACE : QLORA_ERR_ALIGNMENT;
+  if (a.ws_bytes < plan_ws(a.m, a.q->n_out, a.q->k_in, a.r, sms).total) return QLORA_ERR_WORKSPACE;
+  return QLORA_OK;
+}
+
+}  // namespace
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+int32_t qlora_version(void) { return 100; }
+
+const char* qlora_status_string(qlora_status_t s) {
+  switch (s) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument";
+    case QLORA_ERR_SHAPE: return "unsupported shape";
+    case QLORA_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100 (B200)";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_TIMEOUT: return "kernel gave up on a bounded wait";
+  }
+  return "unknown status";
+}
+
+qlora_status_t qlora_nf4_codebook(float out[16]) {
+  if (out == nullptr) return QLORA_ERR_INVALID_ARG;
+  std::memcpy(out, tables().cb, sizeof(float) * 16);
+  return QLORA_OK;
+}
+
+size_t qlora_nf4_bytes(int64_t n_out, int64_t k_in, int32_t dq_group, size_t out[3]) {
+  if (n_out <= 0 || k_in <= 0 || k_in % kBlock != 0 || dq_group != kGroup) return 0;
+  const int64_t nb = n_out * k_in / kBlock;
+  const size_t b0 = static_cast<size_t>(n_out * k_in / 2);
+  const size_t b1 = static_cast<size_t>(nb);
+  const size_t b2 = static_cast<size_t>(cdiv(nb, kGroup)) * sizeof(float);
+  if (out) {
+    out[0] = b0;
+    out[1] = b1;
+    out[2] = b2;
+  }
+  return b0 + b1 + b2;
+}
+
+size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r) {
+  if (m < 0 || n_out <= 0 || k_in <= 0 || r < 1 || r > kMaxRank) return 0;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
+  }
+  cudaGetLastError();
+  return plan_ws(std::max<int64_t>(m, 1), n_out, k_in, r, sms).total;
+}
+
+qlora_status_t qlora_quantize_nf4(const void* w_bf16, const qlora_nf4_t* q, void* stream) {
+  qlora_status_t s = check_nf4(q);
+  if (s != QLORA_OK) return s;
+  if (w_bf16 == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(w_bf16)) return QLORA_ERR_ALIGNMENT;
+  if ((s = device_ready(nullptr)) != QLORA_OK) return s;
+  const int64_t nb = q->n_out * q->k_in / kBlock;
+  QuantParams qp{};
+  std::memcpy(qp.mid, tables().mid, sizeof(qp.mid));
+  const int64_t groups = cdiv(nb, kGroup);
+  if (groups > 0x7FFFFFFF) return QLORA_ERR_SHAPE;
+  k_quantize_nf4<<<static_cast<unsigned>(groups), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(w_bf16), nb, reinterpret_cast<uint32_t*>(q->codes), q->scale_codes,
+      q->absmax, qp);
+  return launch_status();
+}
+
+qlora_status_t qlora_dequantize(const qlora_nf4_t* q, void* w_bf16_out, void* stream) {
+  qlora_status_t s = check_nf4(q);
+  if (s != QLORA_OK) return s;
+  if (w_bf16_out == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(w_bf16_out)) return QLORA_ERR_ALIGNMENT;
+  int sms = 0;
+  if ((s = device_ready(&sms)) != QLORA_OK) return s;
+  const int64_t nwords = q->n_out * q->k_in / 8;
+  DequantParams dp{};
+  std::memcpy(dp.cb, tables().cb, sizeof(dp.cb));
+  const int blocks = static_cast<int>(std::min<int64_t>(cdiv(nwords, 256), int64_t(sms) * 16));
+  k_dequantize_nf4<<<std::max(blocks, 1), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint32_t*>(q->codes), q->scale_codes, q->absmax, nwords,
+      static_cast<uint4*>(w_bf16_out), dp);
+  return launch_status();
+}
+
+qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t m, const void* a,
+                                   const void* b, int32_t r, float alpha, void* y, void* u_out,
+                                   void* ws, size_t ws_bytes, int32_t path, void* stream) {
+  int sms = 0;
+  qlora_status_t s = check_nf4(q);
+  if (s != QLORA_OK) return s;
+  if (path < QLORA_FWD_AUTO || path > QLORA_FWD_GEMV) return QLORA_ERR_INVALID_ARG;
+  if ((s = device_ready(&sms)) != QLORA_OK) return s;
+  const LinearArgs la{q, m, r, alpha, ws, ws_bytes};
+  if ((s = check_linear(la, sms)) != QLORA_OK) return s;
+  if (m == 0) return QLORA_OK;
+  if (x == nullptr || a == nullptr || b == nullptr || y == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(a) || !aligned16(b) || !aligned16(y) || (u_out && !aligned16(u_out)))
+    return QLORA_ERR_ALIGNMENT;
+  if (path == QLORA_FWD_AUTO) path = (m <= kGemvMaxM) ? QLORA_FWD_GEMV : QLORA_FWD_GEMM;
+  if (path == QLORA_FWD_GEMV && m > kGemvMaxM) return QLORA_ERR_SHAPE;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t n = q->n_out, k = q->k_in;
+  const int32_t r64 = r64_of(r);
+  const float sc = alpha / static_cast<float>(r);
+  const WsPlan wp = plan_ws(m, n, k, r, sms);
+  uint8_t* wsb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
+  __nv_bfloat16* u_pad = reinterpret_cast<__nv_bfloat16*>(wsb);
+  __nv_bfloat16* b_pad = reinterpret_cast<__nv_bfloat16*>(wsb + wp.u_pad + wp.v_pad);
+  float* part = reinterpret_cast<float*>(wsb + wp.u_pad + wp.v_pad + wp.b_pad);
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  const auto* ab = static_cast<const __nv_bfloat16*>(a);
+  const auto* bb = static_cast<const __nv_bfloat16*>(b);
+  const __nv_bfloat16* b_use = bb;
+  int64_t ldb = r;
+  if (r % 8 != 0) {
+    k_pad_cols<<<static_cast<unsigned>(std::min<int64_t>(cdiv(n * r64, 256), int64_t(sms) * 8)), 256, 0, st>>>(
+        bb, b_pad, n, r, r64);
+    if ((s = launch_status()) != QLORA_OK) return s;
+    b_use = b_pad;
+    ldb = r64;
+  }
+
+  if (path == QLORA_FWD_GEMV) {
+    LoraDownSmallParams lp{};
+    lp.x = xb;
+    lp.a = ab;
+    lp.u_pad = u_pad;
+    lp.u_out = static_cast<__nv_bfloat16*>(u_out);
+    lp.k = k;
+    lp.m = static_cast<int32_t>(m);
+    lp.r = r;
+    lp.r64 = r64;
+    lp.s = sc;
+    k_lora_down_small<<<r64, 256, 0, st>>>(lp);
+    if ((s = launch_status()) != QLORA_OK) return s;
+    GemvParams gp{};
+    gp.codes = q->codes;
+    gp.q2 = q->scale_codes;
+    gp.smax = q->absmax;
+    gp.x = xb;
+    gp.u = u_pad;
+    gp.b = b_use;
+    gp.y = static_cast<__nv_bfloat16*>(y);
+    gp.n = n;
+    gp.k = k;
+    gp.m = static_cast<int32_t>(m);
+    gp.r = r;
+    gp.r64 = r64;
+    gp.ldb = static_cast<int32_t>(ldb);
+    std::memcpy(gp.cb, tables().cb, sizeof(gp.cb));
+    const unsigned grid = static_cast<unsigned>(cdiv(n, 16));
+    if (m <= 8)
+      k_gemv_nf4<1><<<grid, 256, 0, st>>>(gp);
+    else
+      k_gemv_nf4<2><<<grid, 256, 0, st>>>(gp);
+    return launch_status();
+  }
+
+  // u' = bf16(s x A^T) through the tensor cores (split over K)
+  CUtensorMap m_x_a, m_at, m_x_b, m_u, m_codes;
+  if (!map_bf16(&m_x_a, xb, m, k, k, 128) || !map_bf16(&m_at, ab, r, k, k, static_cast<uint32_t>(r64)))
+    return QLORA_ERR_CUDA;
+  s = lora_product<A_TMA_K, B_TMA_K>(m_x_a, m_at, m, k, r, sc, 0, u_pad, static_cast<__nv_bfloat16*>(u_out),
+                                     nullptr, part, sms, st);
+  if (s != QLORA_OK) return s;
+
+  // y^T tiles: A = restored W (on chip), B = x, plus u' B^T as extra k-tiles
+  if (!map_bf16(&m_x_b, xb, m, k, k, 256) || !map_bf16(&m_u, u_pad, m, r64, r64, 256) ||
+      !map2d(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->codes, static_cast<uint64_t>(k / 2),
+             static_cast<uint64_t>(n), static_cast<uint64_t>(k / 2), 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return QLORA_ERR_CUDA;
+  TcParams p{};
+  p.rows = static_cast<int32_t>(n);
+  p.cols = static_cast<int32_t>(m);
+  p.kt_main = static_cast<int32_t>(k / 64);
+  p.kt_lora = r64 / 64;
+  p.kt_split = p.kt_main;
+  p.q2 = q->scale_codes;
+  p.smax = q->absmax;
+  p.kblocks = k / 64;
+  p.w_rows = n;
+  p.w_cols = k;
+  std::memcpy(p.cb, tables().cb, sizeof(p.cb));
+  p.lora = b_use;
+  p.lora_ld = ldb;
+  p.lora_r = (r % 8 != 0) ? r64 : r;
+  p.out = y;
+  p.ldo = n;
+  const dim3 grid(static_cast<unsigned>(cdiv(n, 128)), static_cast<unsigned>(cdiv(m, 256)), 1);
+  const CUtensorMap z = zero_map();
+  return launch_tc<256, A_DQ_K, B_TMA_K, EPI_BF16_T>(grid, st, z, m_x_b, m_u, m_codes, p);
+}
+
+qlora_status_t qlora_linear_fwd(const qlora_nf4_t* q, const void* x, int64_t m, const void* a, const void* b,
+                                int32_t r, float alpha, void* y, void* u_out, void* ws, size_t ws_bytes,
+                                void* stream) {
+  return qlora_linear_fwd_ex(q, x, m, a, b, r, alpha, y, u_out, ws, ws_bytes, QLORA_FWD_AUTO, stream);
+}
+
+qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void* u, const void* dy, int64_t m,
+                                const void* a, const void* b, int32_t r, float alpha, void* dx, float* da,
+                                float* db, void* ws, size_t ws_bytes, void* stream) {
+  int sms = 0;
+  qlora_status_t s = check_nf4(q);
+  if (s != QLORA_OK) return s;
+  if ((s = device_ready(&sms)) != QLORA_OK) return s;
+  const LinearArgs la{q, m, r, alpha, ws, ws_bytes};
+  if ((s = check_linear(la, sms)) != QLORA_OK) return s;
+  if (x == nullptr || dy == nullptr || a == nullptr || b == nullptr || da == nullptr || db == nullptr)
+    return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(a) || !aligned16(b) || !aligned16(da) || !aligned16(db) ||
+      (dx && !aligned16(dx)) || (u && !aligned16(u)))
+    return QLORA_ERR_ALIGNMENT;
+  const int64_t n = q->n_out, k = q->k_in;
+  if (n % 8 != 0) return QLORA_ERR_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (m == 0) {
+    // no tokens: the gradients are exactly zero
+    if (cudaMemsetAsync(da, 0, static_cast<size_t>(r) * k * sizeof(float), st) != cudaSuccess ||
+        cudaMemsetAsync(db, 0, static_cast<size_t>(n) * r * sizeof(float), st) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
+  const int32_t r64 = r64_of(r);
+  const float sc = alpha / static_cast<float>(r);
+  const WsPlan wp = plan_ws(m, n, k, r, sms);
+  uint8_t* wsb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
+  __nv_bfloat16* u_pad = reinterpret_cast<__nv_bfloat16*>(wsb);
+  __nv_bfloat16* v_pad = reinterpret_cast<__nv_bfloat16*>(wsb + wp.u_pad);
+  __nv_bfloat16* b_pad = reinterpret_cast<__nv_bfloat16*>(wsb + wp.u_pad + wp.v_pad);
+  float* part = reinterpret_cast<float*>(wsb + wp.u_pad + wp.v_pad + wp.b_pad);
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  const auto* ab = static_cast<const __nv_bfloat16*>(a);
+  const auto* bb = static_cast<const __nv_bfloat16*>(b);
+  const auto* dyb = static_cast<const __nv_bfloat16*>(dy);
+  const __nv_bfloat16* b_use = bb;
+  int64_t ldb = r;
+  if (r % 8 != 0) {
+    k_pad_cols<<<static_cast<unsigned>(std::min<int64_t>(cdiv(n * r64, 256), int64_t(sms) * 8)), 256, 0, st>>>(
+        bb, b_pad, n, r, r64);
+    if ((s = launch_status()) != QLORA_OK) return s;
+    b_use = b_pad;
+    ldb = r64;
+  }
+
+  // u' (saved by the forward, padded here when needed, or recomputed)
+  const __nv_bfloat16* u_use = nullptr;
+  int64_t ldu = r64;
+  if (u != nullptr && r % 8 == 0) {
+    u_use = static_cast<const __nv_bfloat16*>(u);
+    ldu = r;
+  } else if (u != nullptr) {
+    k_pad_cols<<<static_cast<unsigned>(std::min<int64_t>(cdiv(m * r64, 256), int64_t(sms) * 8)), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(u), u_pad, m, r, r64);
+    if ((s = launch_status()) != QLORA_OK) return s;
+    u_use = u_pad;
+  } else {
+    CUtensorMap m_x_a, m_at;
+    if (!map_bf16(&m_x_a, xb, m, k, k, 128) || !map_bf16(&m_at, ab, r, k, k, static_cast<uint32_t>(r64)))
+      return QLORA_ERR_CUDA;
+    s = lora_product<A_TMA_K, B_TMA_K>(m_x_a, m_at, m, k, r, sc, 0, u_pad, nullptr, nullptr, part, sms, st);
+    if (s != QLORA_OK) return s;
+    u_use = u_pad;
+  }
+
+  // v' = bf16(s dY B): A = dY (K-major), B = B_lora seen MN-major, reduction over N
+  {
+    CUtensorMap m_dy_a, m_bmn;
+    if (!map_bf16(&m_dy_a, dyb, m, n, n, 128) || !map_bf16(&m_bmn, b_use, n, ldb == r ? r : r64, ldb, 64))
+      return QLORA_ERR_CUDA;
+    s = lora_product<A_TMA_K, B_TMA_MN>(m_dy_a, m_bmn, m, n, r, sc, 0, v_pad, nullptr, nullptr, part, sms, st);
+    if (s != QLORA_OK) return s;
+  }
+
+  // dX^T tiles: A = restored W seen MN-major (reduction over d_out), B = dY,
+  // plus v' A_lora as extra k-tiles
+  if (dx != nullptr) {
+    CUtensorMap m_dy_b, m_v, m_codes;
+    if (!map_bf16(&m_dy_b, dyb, m, n, n, 256) || !map_bf16(&m_v, v_pad, m, r64, r64, 256) ||
+        !map2d(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->codes, static_cast<uint64_t>(k / 2),
+               static_cast<uint64_t>(n), static_cast<uint64_t>(k / 2), 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return QLORA_ERR_CUDA;
+    TcParams p{};
+    p.rows = static_cast<int32_t>(k);
+    p.cols = static_cast<int32_t>(m);
+    p.kt_main = static_cast<int32_t>(cdiv(n, 64));
+    p.kt_lora = r64 / 64;
+    p.kt_split = p.kt_main;
+    p.q2 = q->scale_codes;
+    p.smax = q->absmax;
+    p.kblocks = k / 64;
+    p.w_rows = n;
+    p.w_cols = k;
+    std::memcpy(p.cb, tables().cb, sizeof(p.cb));
+    p.lora = ab;
+    p.lora_ld = k;
+    p.lora_r = r;
+    p.out = dx;
+    p.ldo = k;
+    const dim3 grid(static_cast<unsigned>(cdiv(k, 128)), static_cast<unsigned>(cdiv(m, 256)), 1);
+    const CUtensorMap z = zero_map();
+    s = launch_tc<256, A_DQ_MN, B_TMA_K, EPI_BF16_T>(grid, st, z, m_dy_b, m_v, m_codes, p);
+    if (s != QLORA_OK) return s;
+  }
+
+  // dA^T [K x r] = x^T v'  (A = x seen MN-major, B = v' MN-major, reduction over tokens)
+  {
+    CUtensorMap m_xmn, m_vmn;
+    if (!map_bf16(&m_xmn, xb, m, k, k, 64) || !map_bf16(&m_vmn, v_pad, m, r64, r64, 64)) return QLORA_ERR_CUDA;
+    s = lora_product<A_TMA_MN, B_TMA_MN>(m_xmn, m_vmn, k, m, r, 1.0f, 2, nullptr, nullptr, da, part, sms, st);
+    if (s != QLORA_OK) return s;
+  }
+  // dB [N x r] = dY^T u'  (A = dY seen MN-major, B = u' MN-major)
+  {
+    CUtensorMap m_dymn, m_umn;
+    if (!map_bf16(&m_dymn, dyb, m, n, n, 64) || !map_bf16(&m_umn, u_use, m, ldu == r ? r : r64, ldu, 64))
+      return QLORA_ERR_CUDA;
+    s = lora_product<A_TMA_MN, B_TMA_MN>(m_dymn, m_umn, n, m, r, 1.0f, 1, nullptr, nullptr, db, part, sms, st);
+    if (s != QLORA_OK) return s;
+  }
+  return QLORA_OK;
+}
+
+qlora_status_t qlora_device_status(void* stream, uint32_t* bits) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QLORA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dev_status, sizeof(v)) != cudaSuccess) return QLORA_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (v != 0 && cudaMemcpyToSymbol(g_dev_status, &zero, sizeof(zero)) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (bits) *bits = v;
+  return v ? QLORA_ERR_TIMEOUT : QLORA_OK;
+}
+
+}  // extern "C"

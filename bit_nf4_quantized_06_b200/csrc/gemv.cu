@@ -1,0 +1,228 @@
+// Decode-sized forward (M <= 16 tokens) for sm_100a.
+//
+//   y[m][n] = sum_k x[m][k] w_hat[n][k] + sum_j u'[m][j] B[n][j],
+//   u'      = bf16(s * x A^T)          (k_lora_down_small, launched first)
+//
+// At M <= 16 the forward is a stream over the packed weight: 0.5 byte per
+// weight plus 1/64 byte of scale code, so it is bound by HBM bandwidth as
+// long as restoring a weight costs only a few instructions. Each warp owns
+// 16 weight rows; each lane restores whole 64-weight blocks (one table of 16
+// bf16 values per block, then one byte-permute lookup per weight, see
+// nf4_dev.cuh) straight into the A fragments of mma.sync m16n8k16, with the
+// tokens as the 8-wide N side. Because a dot product may visit k in any
+// order, the lane's 8 consecutive weights are placed into fragment slots in
+// the order they come out of the lookup and x is fetched in the same order,
+// so no shuffle is needed. The eight warps of a CTA split K; their partial
+// fragments are summed in a fixed order in shared memory, and the LoRA term
+// is appended as r/16 further MMA steps of the same accumulator.
+#include "kernels.h"
+#include "nf4_dev.cuh"
+
+namespace qlora {
+
+namespace {
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3},"
+      " {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ld_bf16_pair(const __nv_bfloat16* row, int j, int r) {
+  // (row[j], row[j+1]) with zeros past r; 2-byte loads so any r works
+  const uint16_t* p = reinterpret_cast<const uint16_t*>(row);
+  const uint32_t lo = (j < r) ? p[j] : 0u;
+  const uint32_t hi = (j + 1 < r) ? p[j + 1] : 0u;
+  return lo | (hi << 16);
+}
+
+}  // namespace
+
+template <int NT>
+__global__ void __launch_bounds__(256) k_gemv_nf4(GemvParams p) {
+  constexpr int WARPS = 8;
+  __shared__ float s_red[WARPS][32][NT * 4];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;
+  const int qd = lane & 3;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 16;
+  const int64_t r0 = n0 + g;
+  const int64_t r1 = n0 + g + 8;
+  const bool v0 = r0 < p.n;
+  const bool v1 = r1 < p.n;
+  const int64_t kpr = p.k >> 6;
+  const int64_t nchunks = (kpr + 3) >> 2;
+  const int64_t row_bytes = p.k >> 1;
+
+  float acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[t][i] = 0.0f;
+
+  for (int64_t c = warp; c < nchunks; c += WARPS) {
+    const int64_t kb = c * 4 + qd;  // this lane's block within the row
+    const bool kv = kb < kpr;
+    uint4 a_lo = make_uint4(0, 0, 0, 0), a_hi = a_lo, b_lo = a_lo, b_hi = a_lo;
+    float sh0 = 0.0f, sh1 = 0.0f;
+    if (kv && v0) {
+      const uint8_t* src = p.codes + r0 * row_bytes + kb * 32;
+      a_lo = ldg_stream(src);
+      a_hi = ldg_stream(src + 16);
+      const int64_t bi = r0 * kpr + kb;
+      sh0 = restored_scale(__ldg(p.q2 + bi), __ldg(p.smax + (bi >> 8)));
+    }
+    if (kv && v1) {
+      const uint8_t* src = p.codes + r1 * row_bytes + kb * 32;
+      b_lo = ldg_stream(src);
+      b_hi = ldg_stream(src + 16);
+      const int64_t bi = r1 * kpr + kb;
+      sh1 = restored_scale(__ldg(p.q2 + bi), __ldg(p.smax + (bi >> 8)));
+    }
+    const Nf4Table t0 = make_table(p.cb, sh0);
+    const Nf4Table t1 = make_table(p.cb, sh1);
+    const uint32_t wa[8] = {a_lo.x, a_lo.y, a_lo.z, a_lo.w, a_hi.x, a_hi.y, a_hi.z, a_hi.w};
+    const uint32_t wb[8] = {b_lo.x, b_lo.y, b_lo.z, b_lo.w, b_hi.x, b_hi.y, b_hi.z, b_hi.w};
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      uint32_t ra[4], rb[4];
+      lookup8(t0, wa[w], ra);
+      lookup8(t1, wb[w], rb);
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const int tok = t * 8 + g;
+        uint4 xv = make_uint4(0, 0, 0, 0);
+        if (kv && tok < p.m)
+          xv = __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(tok) * p.k + kb * 64 + 8 * w));
+        // slots: logical k (2qd, 2qd+1) <- weights 4h+0, 4h+1; (2qd+8, 2qd+9) <- 4h+2, 4h+3
+        mma_bf16_16816(acc[t], ra[0], rb[0], ra[1], rb[1], xv.x, xv.y);
+        mma_bf16_16816(acc[t], ra[2], rb[2], ra[3], rb[3], xv.z, xv.w);
+      }
+    }
+  }
+
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s_red[warp][lane][t * 4 + i] = acc[t][i];
+  __syncthreads();
+  if (warp != 0) return;
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float v = 0.0f;
+#pragma unroll
+      for (int wv = 0; wv < WARPS; ++wv) v += s_red[wv][lane][t * 4 + i];
+      acc[t][i] = v;
+    }
+
+  // LoRA term: sum_j u'[tok][j] B[n][j], 16 ranks per MMA step
+  const __nv_bfloat16* brow0 = p.b + (v0 ? r0 : 0) * static_cast<int64_t>(p.ldb);
+  const __nv_bfloat16* brow1 = p.b + (v1 ? r1 : 0) * static_cast<int64_t>(p.ldb);
+  const int rv0 = v0 ? p.r : 0;
+  const int rv1 = v1 ? p.r : 0;
+  for (int j0 = 0; j0 < p.r64; j0 += 16) {
+    const int ja = j0 + 2 * qd;
+    const uint32_t a0 = ld_bf16_pair(brow0, ja, rv0);
+    const uint32_t a1 = ld_bf16_pair(brow1, ja, rv1);
+    const uint32_t a2 = ld_bf16_pair(brow0, ja + 8, rv0);
+    const uint32_t a3 = ld_bf16_pair(brow1, ja + 8, rv1);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const int tok = t * 8 + g;
+      uint32_t b0 = 0, b1 = 0;
+      if (tok < p.m) {
+        const uint32_t* urow = reinterpret_cast<const uint32_t*>(p.u + static_cast<int64_t>(tok) * p.r64);
+        b0 = urow[ja >> 1];
+        b1 = urow[(ja + 8) >> 1];
+      }
+      mma_bf16_16816(acc[t], a0, a1, a2, a3, b0, b1);
+    }
+  }
+
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int tok = t * 8 + 2 * qd;
+    if (v0) {
+      if (tok < p.m) p.y[static_cast<int64_t>(tok) * p.n + r0] = __float2bfloat16_rn(acc[t][0]);
+      if (tok + 1 < p.m) p.y[static_cast<int64_t>(tok + 1) * p.n + r0] = __float2bfloat16_rn(acc[t][1]);
+    }
+    if (v1) {
+      if (tok < p.m) p.y[static_cast<int64_t>(tok) * p.n + r1] = __float2bfloat16_rn(acc[t][2]);
+      if (tok + 1 < p.m) p.y[static_cast<int64_t>(tok + 1) * p.n + r1] = __float2bfloat16_rn(acc[t][3]);
+    }
+  }
+}
+
+template __global__ void k_gemv_nf4<1>(GemvParams);
+template __global__ void k_gemv_nf4<2>(GemvParams);
+
+// u'[m][j] = bf16(s * sum_k x[m][k] A[j][k]) for M <= 16: one CTA per rank j,
+// 256 threads split K in 8-element chunks, fixed-order reduction.
+__global__ void __launch_bounds__(256) k_lora_down_small(LoraDownSmallParams p) {
+  __shared__ float s_part[8][16];
+  const int j = blockIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  float acc[16];
+#pragma unroll
+  for (int m = 0; m < 16; ++m) acc[m] = 0.0f;
+  if (j < p.r) {
+    const int64_t nch = p.k >> 3;
+    const uint4* arow = reinterpret_cast<const uint4*>(p.a + static_cast<int64_t>(j) * p.k);
+    for (int64_t c = threadIdx.x; c < nch; c += blockDim.x) {
+      const uint4 av = __ldg(arow + c);
+      const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+      float af[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        af[2 * i] = __uint_as_float(aw[i] << 16);
+        af[2 * i + 1] = __uint_as_float(aw[i] & 0xFFFF0000u);
+      }
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        if (m < p.m) {
+          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * p.k) + c);
+          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[m] = fmaf(af[2 * i], __uint_as_float(xw[i] << 16), acc[m]);
+            acc[m] = fmaf(af[2 * i + 1], __uint_as_float(xw[i] & 0xFFFF0000u), acc[m]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    float v = acc[m];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    if (lane == 0) s_part[warp][m] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < p.m) {
+    const int m = threadIdx.x;
+    float v = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += s_part[w][m];
+    const __nv_bfloat16 b = __float2bfloat16_rn(j < p.r ? v * p.s : 0.0f);
+    p.u_pad[static_cast<int64_t>(m) * p.r64 + j] = b;
+    if (p.u_out != nullptr && j < p.r) p.u_out[static_cast<int64_t>(m) * p.r + j] = b;
+  }
+}
+
+}  // namespace qlora

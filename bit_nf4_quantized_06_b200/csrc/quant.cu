@@ -1,0 +1,163 @@
+// NF4 blockwise quantizer with double quantization, and the standalone
+// restore, for sm_100a.
+//
+// Quantizer ("48GB GPU Fine-Tuning a 65B Model ...", § "Quantization Keeps
+// the Patterns and Reduces Bits per Number"; «QLoRA는 어떻게 65B 모델을 GPU
+// 한 장에 올렸나», § "메모리 회계"):
+//   s_b   = max |w| over 64 consecutive weights of the row-major matrix
+//   q     = #{ j : fl32(w / s_b) > m_j }   (m_j = fp32 midpoints of the levels;
+//            an exact tie goes to the lower level; s_b == 0 stores level 7)
+//   byte  = (q[2i] << 4) | q[2i+1]
+//   s_max = max s_b over 256 consecutive blocks (the last group may be short)
+//   q2    = min(255, rint_even(fl32(256 * s_b / s_max)))   (0 if s_max == 0)
+//
+// One CTA of 256 threads owns one double-quantization group (256 blocks,
+// 16384 weights, 32 KB of bf16): every thread loads 8 x 16 B with fully
+// coalesced warp accesses (lane l reads bytes [16 l, 16 l + 16) of each
+// 512-byte warp slice), the 8 lanes that share a block reduce its absmax
+// with xor shuffles, the group maximum goes through shared memory, and each
+// 8-weight chunk is encoded and written back as one 32-bit word, again
+// coalesced. W is read exactly once; codes, scale codes and s_max are
+// written exactly once.
+#include "ptx.cuh"
+#include "nf4_dev.cuh"
+#include "kernels.h"
+
+namespace qlora {
+
+__device__ unsigned int g_dev_status = 0;
+
+namespace {
+
+__device__ __forceinline__ uint32_t abs_bits_max(uint4 v) {
+  // bf16 magnitudes compare like unsigned integers once the sign is cleared
+  uint32_t m = 0;
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m = max(m, w[i] & 0x7FFFu);
+    m = max(m, (w[i] >> 16) & 0x7FFFu);
+  }
+  return m;
+}
+
+__device__ __forceinline__ uint32_t encode_one(float w, float s, const float* mid) {
+  if (s == 0.0f) return 7u;
+  const float x = __fdiv_rn(w, s);
+  uint32_t q = (x > mid[7]) ? 8u : 0u;
+  q += (x > mid[q + 3]) ? 4u : 0u;
+  q += (x > mid[q + 1]) ? 2u : 0u;
+  q += (x > mid[q]) ? 1u : 0u;
+  return q;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(256) k_quantize_nf4(const uint4* __restrict__ w,
+                                                      int64_t nb, uint32_t* __restrict__ codes,
+                                                      uint8_t* __restrict__ q2,
+                                                      float* __restrict__ smax, QuantParams qp) {
+  __shared__ float s_mid[16];
+  __shared__ uint32_t s_wmax[8];
+  const int tid = threadIdx.x;
+  if (tid < 16) s_mid[tid] = qp.mid[tid];
+
+  const int64_t g = blockIdx.x;
+  const int64_t b0 = g * 256;
+  const int nblk = static_cast<int>(nb - b0 < 256 ? nb - b0 : 256);
+  const int64_t chunk0 = b0 * 8;  // 8 chunks of 8 weights per block
+
+  uint4 v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int bi = (tid >> 3) + 32 * i;
+    v[i] = (bi < nblk) ? __ldcs(w + chunk0 + tid + 256 * i) : make_uint4(0, 0, 0, 0);
+  }
+
+  uint32_t am[8];
+  uint32_t gm = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint32_t m = abs_bits_max(v[i]);
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+    am[i] = m;
+    gm = max(gm, m);
+  }
+  gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 8));
+  gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 16));
+  if ((tid & 31) == 0) s_wmax[tid >> 5] = gm;
+  __syncthreads();
+  uint32_t gmax = s_wmax[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) gmax = max(gmax, s_wmax[i]);
+  const float s_max = __uint_as_float(gmax << 16);
+  if (tid == 0) smax[g] = s_max;
+
+  if ((tid & 7) == 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int bi = (tid >> 3) + 32 * i;
+      if (bi < nblk) {
+        uint32_t code = 0;
+        if (s_max != 0.0f) {
+          const float s = __uint_as_float(am[i] << 16);
+          const float ratio = __fdiv_rn(256.0f * s, s_max);
+          code = static_cast<uint32_t>(min(255, __float2int_rn(ratio)));
+        }
+        q2[b0 + bi] = static_cast<uint8_t>(code);
+      }
+    }
+  }
+
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int bi = (tid >> 3) + 32 * i;
+    if (bi < nblk) {
+      const float s = __uint_as_float(am[i] << 16);
+      const uint32_t ww[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        // bf16 pair j holds elements 2j (low half) and 2j+1 (high half)
+        const float e0 = __uint_as_float(ww[j] << 16);
+        const float e1 = __uint_as_float(ww[j] & 0xFFFF0000u);
+        const uint32_t q0 = encode_one(e0, s, s_mid);
+        const uint32_t q1 = encode_one(e1, s, s_mid);
+        word |= ((q0 << 4) | q1) << (8 * j);
+      }
+      codes[chunk0 + tid + 256 * i] = word;
+    }
+  }
+}
+
+// Restore: one thread per 8 weights (one 32-bit code word -> one 16-byte
+// store). Grid-stride over all words.
+__global__ void __launch_bounds__(256) k_dequantize_nf4(const uint32_t* __restrict__ codes,
+                                                        const uint8_t* __restrict__ q2,
+                                                        const float* __restrict__ smax,
+                                                        int64_t nwords, uint4* __restrict__ out,
+                                                        DequantParams dp) {
+  __shared__ float s_cb[16];
+  if (threadIdx.x < 16) s_cb[threadIdx.x] = dp.cb[threadIdx.x];
+  __syncthreads();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nwords;
+       i += stride) {
+    const int64_t b = i >> 3;
+    const float s_hat = restored_scale(__ldg(q2 + b), __ldg(smax + (b >> 8)));
+    const uint32_t w = __ldcs(codes + i);
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t byte = (w >> (8 * j)) & 0xFFu;
+      const float v0 = __fmul_rn(s_cb[byte >> 4], s_hat);
+      const float v1 = __fmul_rn(s_cb[byte & 15u], s_hat);
+      o[j] = pack_bf16x2(v0, v1);
+    }
+    __stcs(out + i, make_uint4(o[0], o[1], o[2], o[3]));
+  }
+}
+
+}  // namespace qlora

@@ -1,0 +1,160 @@
+/*
+ * qlora.h — C ABI of the B200 (sm_100a) QLoRA NF4 + LoRA quantized linear.
+ *
+ * The operation, as the sources state it:
+ *
+ *   h = dequant(W_NF4, c_block) x + (alpha/r) B A x
+ *     «QLoRA는 어떻게 65B 모델을 GPU 한 장에 올렸나» (iq-universe blog),
+ *     § "QLoRA의 수식: 두 항의 결합".
+ *   Storage: blocks of 64 weights, one absmax scale per block, each weight a
+ *   4-bit index of the nearest normal-quantile level; the scales themselves
+ *   re-quantized to 8 bits ("double quantization"), about 4.13 bits/param;
+ *   weights restored to bf16 just before each matmul.
+ *     "48GB GPU Fine-Tuning a 65B Model: Where QLoRA Saves GPU Memory",
+ *     § "Quantization Keeps the Patterns and Reduces Bits per Number";
+ *     «QLoRA는 …», § "메모리 회계: 세 겹의 최적화" (restore formula
+ *     c(q) * q2/256 * s_max, error at most s_max/256).
+ *   Backward: W is frozen, gradients flow through the restored W to x and to
+ *   A and B only.
+ *     «QLoRA는 …», § "명제 1 · QLoRA Backward Unbiasedness";
+ *     "48GB GPU …", § "QLoRA Puts the Two Methods in Different Places".
+ *
+ * Notation (row-major everywhere, tokens in rows):
+ *   W  [N x K] bf16   frozen base weight (N = d_out, K = d_in, K % 64 == 0)
+ *   x  [M x K] bf16   input tokens
+ *   A  [r x K] bf16   LoRA down projection
+ *   B  [N x r] bf16   LoRA up projection
+ *   s = alpha / r
+ *   y  = x W_hat^T + s (x A^T) B^T                         [M x N] bf16
+ *   u' = bf16(s * x A^T)                                    [M x r] bf16
+ *   dX = dY W_hat + s (dY B) A                              [M x K] bf16
+ *   dA = s (dY B)^T x                                       [r x K] fp32
+ *   dB = s dY^T (x A^T)                                     [N x r] fp32
+ *
+ * Stored format (readings where the sources are silent):
+ *   codes       [N x K/2] u8   byte i of a row = (q[2i] << 4) | q[2i+1]
+ *   scale_codes [N*K/64]  u8   q2 = min(255, rint(fl32(256 * absmax / s_max)))
+ *   absmax      [ceil(N*K/64 / 256)] fp32   s_max per group of 256
+ *                              consecutive blocks (row-major block order)
+ *   restore:    w_hat = bf16_rne(fl32(c[q] * (fl32(q2 * s_max) * 2^-8)))
+ *
+ * Conventions for every call:
+ *   - Memory is owned by the CALLER. The library never allocates, frees or
+ *     synchronises; every device pointer must be 16-byte aligned.
+ *   - Calls are asynchronous and ordered on the given CUDA stream
+ *     (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *   - Argument, shape, alignment and device errors are returned
+ *     synchronously, before anything is launched. A failed launch returns
+ *     QLORA_ERR_CUDA. No C++ exception crosses the ABI.
+ *   - Kernels never wait without a bound: a pipeline wait that exceeds about
+ *     two seconds ends the kernel and sets a device status bit that
+ *     qlora_device_status() reports as QLORA_ERR_TIMEOUT.
+ *   - Inputs must be finite; results for non-finite weights are unspecified.
+ */
+#ifndef QLORA_H_
+#define QLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, alpha/r not finite   */
+  QLORA_ERR_SHAPE = 2,             /* K % 64 != 0, empty where not allowed, r range */
+  QLORA_ERR_ALIGNMENT = 3,         /* a device pointer not 16-byte aligned          */
+  QLORA_ERR_WORKSPACE = 4,         /* ws too small (see qlora_workspace_bytes)      */
+  QLORA_ERR_UNSUPPORTED_DEVICE = 5,/* current device is not sm_100                 */
+  QLORA_ERR_CUDA = 6,              /* a CUDA runtime / launch error                 */
+  QLORA_ERR_TIMEOUT = 7            /* a kernel gave up on a bounded wait            */
+} qlora_status_t;
+
+/* Packed NF4 weight with double-quantized scales. All pointers are device
+ * pointers owned by the caller; sizes from qlora_nf4_bytes(). */
+typedef struct {
+  int64_t n_out;         /* N rows (d_out)                                     */
+  int64_t k_in;          /* K columns (d_in), K % 64 == 0                      */
+  int32_t block;         /* weights per absmax block: must be 64               */
+  int32_t dq_group;      /* blocks per double-quantization group: must be 256 */
+  uint8_t *codes;        /* N*K/2 bytes                                        */
+  uint8_t *scale_codes;  /* N*K/64 bytes                                       */
+  float *absmax;         /* ceil(N*K/64/256) floats: the group constants s_max */
+} qlora_nf4_t;
+
+/* Forward path selection for qlora_linear_fwd_ex. AUTO takes the decode GEMV
+ * for m <= 16 and the tensor-core GEMM otherwise. */
+typedef enum { QLORA_FWD_AUTO = 0, QLORA_FWD_GEMM = 1, QLORA_FWD_GEMV = 2 } qlora_fwd_path_t;
+
+/* Byte sizes of the three stored arrays; returns their sum (0 on bad shape).
+ * out may be NULL. Host only, no device work. */
+QLORA_API size_t qlora_nf4_bytes(int64_t n_out, int64_t k_in, int32_t dq_group, size_t out[3]);
+
+/* The library's own fp32 NF4 table (16 ascending levels in [-1, 1] with an
+ * exact zero at index 7), computed on the host by Newton iteration on erfc:
+ * 8 positive levels Phi^-1(d + j(1/2 - d)/8), j = 0..7, 7 negative levels
+ * -Phi^-1(d + j(1/2 - d)/7), j = 0..6, and 0, d = ((1-1/30)+(1-1/32))/2,
+ * divided by Phi^-1(d). Host only. */
+QLORA_API qlora_status_t qlora_nf4_codebook(float out[16]);
+
+/* Quantize a bf16 weight W [N x K] (device) into q (device buffers). One pass
+ * over W: per-block absmax, nearest-level encode, nibble packing, and the
+ * 8-bit double quantization of the scales. Bit-exact with the definition in
+ * the stored-format paragraph above. */
+QLORA_API qlora_status_t qlora_quantize_nf4(const void *w_bf16, const qlora_nf4_t *q, void *stream);
+
+/* Restore W_hat [N x K] bf16 (device) from q. Bit-exact. */
+QLORA_API qlora_status_t qlora_dequantize(const qlora_nf4_t *q, void *w_bf16_out, void *stream);
+
+/* Workspace bytes that qlora_linear_fwd / _bwd need for these sizes (an
+ * upper bound that covers both calls and every forward path). */
+QLORA_API size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r);
+
+/* Forward: y [m x N] = x W_hat^T + s (x A^T) B^T, bf16 out, fp32 accumulate.
+ * x [m x K], A [r x K], B [N x r] bf16 (device); 1 <= r <= 256; m >= 0
+ * (m == 0 is a no-op). u_out [m x r] bf16 receives u' = bf16(s x A^T) for
+ * the backward pass; it may be NULL. ws/ws_bytes: caller-owned scratch. */
+QLORA_API qlora_status_t qlora_linear_fwd(const qlora_nf4_t *q, const void *x_bf16, int64_t m,
+                                const void *a_bf16, const void *b_bf16, int32_t r, float alpha,
+                                void *y_bf16, void *u_out_bf16, void *ws, size_t ws_bytes,
+                                void *stream);
+
+/* As qlora_linear_fwd, with the forward path chosen explicitly. */
+QLORA_API qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t *q, const void *x_bf16, int64_t m,
+                                   const void *a_bf16, const void *b_bf16, int32_t r,
+                                   float alpha, void *y_bf16, void *u_out_bf16, void *ws,
+                                   size_t ws_bytes, int32_t path, void *stream);
+
+/* Backward: dX [m x K] bf16 (may be NULL to skip), dA [r x K] fp32 and
+ * dB [N x r] fp32 (overwritten, not accumulated). u_bf16 is the u' that the
+ * forward produced ([m x r], may be NULL: then it is recomputed). No gradient
+ * into W. N % 8 == 0 is required here (dY rows are read by TMA). */
+QLORA_API qlora_status_t qlora_linear_bwd(const qlora_nf4_t *q, const void *x_bf16, const void *u_bf16,
+                                const void *dy_bf16, int64_t m, const void *a_bf16,
+                                const void *b_bf16, int32_t r, float alpha, void *dx_bf16,
+                                float *da, float *db, void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronises `stream`, then reads and clears the device status word of the
+ * current device. Returns QLORA_OK, QLORA_ERR_TIMEOUT (a kernel gave up on a
+ * bounded wait; *bits, if non-NULL, gets which role), or QLORA_ERR_CUDA. */
+QLORA_API qlora_status_t qlora_device_status(void *stream, uint32_t *bits);
+
+/* Static description of a status code. */
+QLORA_API const char *qlora_status_string(qlora_status_t s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+QLORA_API int32_t qlora_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H_ */

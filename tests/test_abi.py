@@ -1,0 +1,80 @@
+"""The C-ABI library loads, exports every symbol include/qlora.h declares, and its
+host-only logic behaves (no GPU needed: nothing here launches a kernel)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import nf4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora.h")
+
+
+@pytest.fixture(scope="module")
+def q():
+    import bit_nf4_quantized_06_b200 as q
+    return q
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"QLORA_API\s+[\w\s\*]*?\b(qlora_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("qlora_quantize_nf4", "qlora_dequantize", "qlora_linear_fwd", "qlora_linear_bwd"):
+        assert name in syms
+
+
+def test_every_declared_symbol_is_exported(q):
+    lib = ctypes.CDLL(q.LIB_PATH)
+    missing = [s for s in declared_symbols() if not hasattr(lib, s)]
+    assert not missing, missing
+
+
+def test_codebook_bit_equal_to_oracle(q):
+    # the library computes its table by Newton iteration on erfc; the oracle
+    # uses statistics.NormalDist: the two fp32 tables must agree bit for bit
+    lib_cb = np.array(q.qlora_nf4_codebook(), dtype=np.float32)
+    assert np.array_equal(lib_cb.view(np.uint32), nf4.codebook().view(np.uint32))
+
+
+def test_nf4_bytes_matches_storage_format(q):
+    for n, k in ((512, 512), (11008, 4096), (37, 192), (8192, 22016)):
+        assert q.qlora_nf4_bytes(n, k) == nf4.storage_bytes(n, k, dq=True)
+    with pytest.raises(q.QloraError):
+        q.qlora_nf4_bytes(16, 100)      # K % 64 != 0
+    with pytest.raises(q.QloraError):
+        q.qlora_nf4_bytes(16, 64, 128)  # only groups of 256
+
+
+def test_status_strings_and_version(q):
+    assert q.qlora_status_string(0) == "ok"
+    assert "aligned" in q.qlora_status_string(3)
+    assert q.qlora_version() >= 100
+
+
+def test_workspace_bytes_positive_and_monotone(q):
+    a = q.qlora_workspace_bytes(16, 512, 512, 8)
+    b = q.qlora_workspace_bytes(4096, 11008, 4096, 64)
+    assert 0 < a < b
+    assert q.qlora_workspace_bytes(16, 512, 512, 0) == 0
+    assert q.qlora_workspace_bytes(16, 512, 512, 257) == 0
+
+
+def test_argument_validation_before_any_launch(q):
+    lib = q.lib
+    s = q.Nf4Struct(512, 512, 64, 256, 0, 0, 0)           # null buffers
+    assert lib.qlora_quantize_nf4(ctypes.c_void_p(16), ctypes.byref(s), None) == 1
+    s = q.Nf4Struct(512, 500, 64, 256, 16, 16, 16)       # K % 64 != 0
+    assert lib.qlora_dequantize(ctypes.byref(s), ctypes.c_void_p(16), None) == 2
+    s = q.Nf4Struct(512, 512, 32, 256, 16, 16, 16)       # block must be 64
+    assert lib.qlora_dequantize(ctypes.byref(s), ctypes.c_void_p(16), None) == 1
+    s = q.Nf4Struct(512, 512, 64, 256, 17, 16, 16)       # misaligned codes
+    assert lib.qlora_dequantize(ctypes.byref(s), ctypes.c_void_p(16), None) == 3
+    assert lib.qlora_nf4_codebook(None) == 1

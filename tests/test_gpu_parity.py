@@ -1,0 +1,310 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+* quantizer and standalone restore: bit-exact (codes, scale codes, s_max, bf16 W_hat);
+* forward / backward: relative Frobenius error <= 5e-3 per output against the
+  fp64 oracle evaluated on the oracle's own W_hat and the same bf16 inputs;
+* the restore inside the GEMMs is bit-exact too: x = I with B = 0 gives
+  W_hat^T exactly, dY = I with B = 0 gives W_hat exactly.
+
+After every test the device status word must be clear (no kernel gave up on
+a bounded wait).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import bf16 as obf16
+from oracle import linear, nf4
+
+pytestmark = pytest.mark.gpu
+
+TOL = 5e-3
+
+
+@pytest.fixture(scope="module")
+def q():
+    import bit_nf4_quantized_06_b200 as q
+    return q
+
+
+@pytest.fixture(autouse=True)
+def _status_clear(q):
+    yield
+    st, bits = q.qlora_device_status()
+    assert st == 0 and bits == 0, f"device status {st} bits {bits:#x}"
+
+
+def _np(t):
+    return t.detach().cpu().float().numpy()
+
+
+def _oracle_quant(w_cpu_bf16):
+    return nf4.quantize(w_cpu_bf16.float().numpy())
+
+
+def _oracle_what(o):
+    return nf4.dequantize(o["codes"], o["q2"], o["smax"])
+
+
+def _bits(t):
+    return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+# --------------------------------------------------------------------------- quantizer / restore
+
+QUANT_SHAPES = [
+    (512, 512, False, 0),
+    (37, 192, False, 1),        # 111 blocks: a short last group, rows not a multiple of anything
+    (64, 4096, True, 2),        # outlier blocks
+    (3, 64, False, 3),          # a single block per row
+    (1024, 1088, True, 4),      # 17 blocks per row: groups straddle rows
+]
+
+
+@pytest.mark.parametrize("n,k,outl,seed", QUANT_SHAPES)
+def test_quantize_bit_exact(q, n, k, outl, seed):
+    w = synth.weight(n, k, seed=seed, outliers=outl)
+    if n >= 3:
+        w[1, : min(k, 128)] = 0          # zero blocks
+        w[2, :64] = -w[2, :64]
+    o = _oracle_quant(w)
+    qw = q.qlora_quantize_nf4(w.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(qw.codes.cpu().numpy(), o["codes"].ravel())
+    assert np.array_equal(qw.scale_codes.cpu().numpy(), o["q2"])
+    assert np.array_equal(qw.absmax.cpu().numpy().view(np.uint32), o["smax"].view(np.uint32))
+
+
+@pytest.mark.parametrize("n,k,outl,seed", QUANT_SHAPES)
+def test_dequantize_bit_exact(q, n, k, outl, seed):
+    w = synth.weight(n, k, seed=seed, outliers=outl)
+    o = _oracle_quant(w)
+    qw = q.qlora_quantize_nf4(w.cuda())
+    wh = q.qlora_dequantize(qw)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(wh), nf4.dequantize_bits(o["codes"], o["q2"], o["smax"]))
+
+
+def test_quantize_full_size_7b_mlp(q):
+    p = synth.MLP7B
+    w = synth.weight(p.n, p.k)
+    o = _oracle_quant(w)
+    qw = q.qlora_quantize_nf4(w.cuda())
+    wh = q.qlora_dequantize(qw)
+    torch.cuda.synchronize()
+    assert np.array_equal(qw.codes.cpu().numpy(), o["codes"].ravel())
+    assert np.array_equal(qw.scale_codes.cpu().numpy(), o["q2"])
+    assert np.array_equal(qw.absmax.cpu().numpy().view(np.uint32), o["smax"].view(np.uint32))
+    assert np.array_equal(_bits(wh), nf4.dequantize_bits(o["codes"], o["q2"], o["smax"]))
+
+
+@pytest.mark.parametrize("p", [synth.GATE65B, synth.DOWN65B], ids=lambda p: p.name)
+def test_quantize_full_size_65b_sampled_rows(q, p):
+    # rows [r0, r0 + R) that start on a group boundary hold whole groups, so
+    # the oracle on those rows alone reproduces their codes and constants
+    w = synth.weight(p.n, p.k, outliers=True)
+    qw = q.qlora_quantize_nf4(w.cuda())
+    torch.cuda.synchronize()
+    kb = p.k // 64
+    step = 256 // np.gcd(kb, 256)                   # rows per whole number of groups
+    rows = max(step, 32 - 32 % step)
+    for r0 in (0, (p.n // 2) // step * step, (p.n - rows) // step * step):
+        o = nf4.quantize(w[r0:r0 + rows].float().numpy())
+        codes = qw.codes.view(p.n, p.k // 2)[r0:r0 + rows].cpu().numpy()
+        assert np.array_equal(codes, o["codes"])
+        b0 = r0 * kb
+        assert np.array_equal(qw.scale_codes[b0:b0 + rows * kb].cpu().numpy(), o["q2"])
+        g0 = b0 // 256
+        assert np.array_equal(qw.absmax[g0:g0 + o["smax"].size].cpu().numpy().view(np.uint32),
+                              o["smax"].view(np.uint32))
+
+
+# --------------------------------------------------------------------------- forward
+
+def _problem(n, k, m, r, seed=0, outliers=False):
+    t = {
+        "w": synth.weight(n, k, seed=seed, outliers=outliers),
+        "x": synth.tokens(m, k, seed=seed),
+        "a": synth.lora_a(r, k, seed=seed),
+        "b": synth.lora_b(n, r, seed=seed),
+        "dy": synth.grad_out(m, n, seed=seed),
+    }
+    return t
+
+
+FWD_CASES = [
+    # n, k, m, r, path
+    (512, 512, 16, 8, "gemm"),
+    (512, 512, 16, 8, "gemv"),
+    (512, 512, 300, 8, "gemm"),      # ragged token tail
+    (200, 192, 37, 64, "gemm"),      # ragged rows, 3 k-tiles
+    (256, 256, 129, 100, "gemm"),    # r not a multiple of 8 (padded copies)
+    (384, 1024, 513, 256, "gemm"),   # largest rank
+    (4096, 4096, 1, 64, "gemv"),     # decode shape
+    (1000, 512, 3, 12, "gemv"),
+    (1000, 512, 9, 12, "gemv"),      # two token groups
+]
+
+
+@pytest.mark.parametrize("n,k,m,r,path", FWD_CASES)
+def test_forward_parity(q, n, k, m, r, path):
+    alpha = 16.0
+    t = _problem(n, k, m, r, seed=n + k + m)
+    o = _oracle_quant(t["w"])
+    w_hat = _oracle_what(o)
+    y_ref, u_ref = linear.forward(_np(t["x"]), w_hat, _np(t["a"]), _np(t["b"]), alpha / r)
+    qw = q.qlora_quantize_nf4(t["w"].cuda())
+    mode = q.FWD_GEMM if path == "gemm" else q.FWD_GEMV
+    y, u = q.qlora_linear_fwd_ex(qw, t["x"].cuda(), t["a"].cuda(), t["b"].cuda(), alpha, path=mode)
+    torch.cuda.synchronize()
+    assert linear.rel_fro(_np(y), y_ref) <= TOL
+    assert linear.rel_fro(_np(u), (alpha / r) * u_ref) <= TOL
+
+
+def test_forward_gemm_restores_w_exactly(q):
+    # x = I (tokens = K), B = 0: y[m][n] = W_hat[n][m] with no rounding left
+    n, k, r = 320, 192, 16
+    w = synth.weight(n, k, seed=5)
+    o = _oracle_quant(w)
+    qw = q.qlora_quantize_nf4(w.cuda())
+    x = torch.eye(k, dtype=torch.bfloat16)
+    a = synth.lora_a(r, k)
+    b = torch.zeros((n, r), dtype=torch.bfloat16)
+    y, _ = q.qlora_linear_fwd_ex(qw, x.cuda(), a.cuda(), b.cuda(), 16.0, path=q.FWD_GEMM)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(y).T, nf4.dequantize_bits(o["codes"], o["q2"], o["smax"]))
+
+
+def test_forward_gemv_restores_w_exactly(q):
+    n, k, r = 256, 512, 8
+    w = synth.weight(n, k, seed=6)
+    o = _oracle_quant(w)
+    qw = q.qlora_quantize_nf4(w.cuda())
+    ref = nf4.dequantize_bits(o["codes"], o["q2"], o["smax"])
+    b = torch.zeros((n, r), dtype=torch.bfloat16)
+    a = synth.lora_a(r, k)
+    for k0 in (0, 77, 511):
+        x = torch.zeros((3, k), dtype=torch.bfloat16)
+        x[0, k0] = 1
+        x[2, (k0 + 5) % k] = 1
+        y, _ = q.qlora_linear_fwd_ex(qw, x.cuda(), a.cuda(), b.cuda(), 16.0, path=q.FWD_GEMV)
+        torch.cuda.synchronize()
+        yb = _bits(y)
+        assert np.array_equal(yb[0], ref[:, k0])
+        assert np.array_equal(yb[2], ref[:, (k0 + 5) % k])
+        assert np.all(yb[1] == 0)
+
+
+def test_forward_w_zero_is_lora_only(q):
+    n, k, m, r = 256, 256, 64, 32
+    t = _problem(n, k, m, r, seed=11)
+    w = torch.zeros((n, k), dtype=torch.bfloat16)
+    qw = q.qlora_quantize_nf4(w.cuda())
+    y, _ = q.qlora_linear_fwd_ex(qw, t["x"].cuda(), t["a"].cuda(), t["b"].cuda(), 8.0, path=q.FWD_GEMM)
+    torch.cuda.synchronize()
+    y_ref, _ = linear.forward(_np(t["x"]), np.zeros((n, k)), _np(t["a"]), _np(t["b"]), 8.0 / r)
+    assert linear.rel_fro(_np(y), y_ref) <= TOL
+
+
+def test_forward_empty_tokens_is_noop(q):
+    n, k, r = 128, 128, 8
+    qw = q.qlora_quantize_nf4(synth.weight(n, k).cuda())
+    x = torch.empty((0, k), dtype=torch.bfloat16, device="cuda")
+    y, u = q.qlora_linear_fwd(qw, x, synth.lora_a(r, k).cuda(), synth.lora_b(n, r).cuda(), 16.0,
+                              ws=torch.empty(256, dtype=torch.uint8, device="cuda"))
+    assert y.shape == (0, n)
+
+
+# --------------------------------------------------------------------------- backward
+
+BWD_CASES = [
+    (512, 512, 16, 8),
+    (512, 512, 300, 8),
+    (200, 192, 37, 64),
+    (256, 256, 129, 100),
+    (384, 1024, 513, 256),
+    (1000, 512, 70, 12),
+]
+
+
+@pytest.mark.parametrize("n,k,m,r", BWD_CASES)
+@pytest.mark.parametrize("with_u", [True, False])
+def test_backward_parity(q, n, k, m, r, with_u):
+    alpha = 16.0
+    s = alpha / r
+    t = _problem(n, k, m, r, seed=3 * n + k + m)
+    o = _oracle_quant(t["w"])
+    w_hat = _oracle_what(o)
+    dx_ref, da_ref, db_ref = linear.backward(_np(t["x"]), _np(t["dy"]), w_hat, _np(t["a"]), _np(t["b"]), s)
+    qw = q.qlora_quantize_nf4(t["w"].cuda())
+    x, a, b, dy = (t[k_].cuda() for k_ in ("x", "a", "b", "dy"))
+    _, u = q.qlora_linear_fwd_ex(qw, x, a, b, alpha, path=q.FWD_GEMM)
+    dx, da, db = q.qlora_linear_bwd(qw, x, u if with_u else None, dy, a, b, alpha)
+    torch.cuda.synchronize()
+    assert linear.rel_fro(_np(dx), dx_ref) <= TOL
+    assert linear.rel_fro(_np(da), da_ref) <= TOL
+    assert linear.rel_fro(_np(db), db_ref) <= TOL
+
+
+def test_backward_dx_restores_w_exactly(q):
+    # dY = I (tokens = N rows), B = 0: dX[m] = W_hat[m] exactly
+    n, k, r = 192, 320, 16
+    w = synth.weight(n, k, seed=7)
+    o = _oracle_quant(w)
+    qw = q.qlora_quantize_nf4(w.cuda())
+    dy = torch.eye(n, dtype=torch.bfloat16)
+    x = synth.tokens(n, k)
+    a = synth.lora_a(r, k)
+    b = torch.zeros((n, r), dtype=torch.bfloat16)
+    dx, da, db = q.qlora_linear_bwd(qw, x.cuda(), None, dy.cuda(), a.cuda(), b.cuda(), 16.0)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(dx), nf4.dequantize_bits(o["codes"], o["q2"], o["smax"]))
+    assert torch.count_nonzero(da).item() == 0        # B = 0 -> no gradient into A
+
+
+def test_backward_requires_n_multiple_of_8(q):
+    n, k, m, r = 100, 128, 16, 8
+    t = _problem(n, k, m, r)
+    qw = q.qlora_quantize_nf4(t["w"].cuda())
+    with pytest.raises(q.QloraError):
+        q.qlora_linear_bwd(qw, t["x"].cuda(), None, t["dy"].cuda(), t["a"].cuda(), t["b"].cuda(), 16.0)
+
+
+# --------------------------------------------------------------------------- full size (bench launch shape)
+
+def test_full_size_7b_mlp_fwd_bwd_sampled(q):
+    p = synth.MLP7B
+    t = synth.make(p)
+    o = _oracle_quant(t["w"])
+    w_hat = _oracle_what(o).astype(np.float64)
+    qw = q.qlora_quantize_nf4(t["w"].cuda())
+    x, a, b, dy = (t[k_].cuda() for k_ in ("x", "a", "b", "dy"))
+    y, u = q.qlora_linear_fwd(qw, x, a, b, p.alpha)
+    dx, da, db = q.qlora_linear_bwd(qw, x, u, dy, a, b, p.alpha)
+    torch.cuda.synchronize()
+    s = p.scale
+    xn, an, bn, dyn = (_np(t[k_]).astype(np.float64) for k_ in ("x", "a", "b", "dy"))
+    rows = np.array([0, 1, 255, 256, 1000, 2047, 3071, 4095])
+    y_ref = xn[rows] @ w_hat.T + s * (xn[rows] @ an.T) @ bn.T
+    assert linear.rel_fro(_np(y)[rows], y_ref) <= TOL
+    v = dyn @ bn
+    dx_ref = dyn[rows] @ w_hat + s * v[rows] @ an
+    assert linear.rel_fro(_np(dx)[rows], dx_ref) <= TOL
+    da_ref = s * (v.T @ xn)
+    db_ref = s * (dyn.T @ (xn @ an.T))
+    assert linear.rel_fro(_np(da), da_ref) <= TOL
+    assert linear.rel_fro(_np(db), db_ref) <= TOL
+
+
+def test_full_size_decode_gemv(q):
+    p = synth.DECODE
+    t = synth.make(p)
+    o = _oracle_quant(t["w"])
+    w_hat = _oracle_what(o)
+    y_ref, _ = linear.forward(_np(t["x"]), w_hat, _np(t["a"]), _np(t["b"]), p.scale)
+    qw = q.qlora_quantize_nf4(t["w"].cuda())
+    y, _ = q.qlora_linear_fwd(qw, t["x"].cuda(), t["a"].cuda(), t["b"].cuda(), p.alpha)
+    torch.cuda.synchronize()
+    assert linear.rel_fro(_np(y), y_ref) <= TOL
