@@ -10,7 +10,8 @@ Functions carry the C names:
 
     qlora_nf4_bytes, qlora_nf4_codebook, qlora_quantize_nf4, qlora_dequantize,
     qlora_workspace_bytes, qlora_linear_fwd, qlora_linear_fwd_ex,
-    qlora_linear_bwd, qlora_device_status, qlora_status_string, qlora_version
+    qlora_linear_bwd, qlora_device_status, qlora_status_string, qlora_version,
+    qlora_launch_count
 """
 
 import ctypes
@@ -20,14 +21,14 @@ __all__ = [
     "LIB_PATH", "lib", "QloraError", "NF4Weight", "Nf4Struct",
     "qlora_nf4_bytes", "qlora_nf4_codebook", "qlora_quantize_nf4", "qlora_dequantize",
     "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_fwd_ex", "qlora_linear_bwd",
-    "qlora_device_status", "qlora_status_string", "qlora_version",
+    "qlora_device_status", "qlora_status_string", "qlora_version", "qlora_launch_count",
     "FWD_AUTO", "FWD_GEMM", "FWD_GEMV",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlora.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m bit_nf4_quantized_06_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python bit_nf4_quantized_06_b200/build.py` "
         "(there is no CPU or Python fallback)")
 
 lib = ctypes.CDLL(LIB_PATH)
@@ -76,6 +77,8 @@ lib.qlora_status_string.argtypes = [ctypes.c_int]
 lib.qlora_status_string.restype = ctypes.c_char_p
 lib.qlora_version.argtypes = []
 lib.qlora_version.restype = _i32
+lib.qlora_launch_count.argtypes = []
+lib.qlora_launch_count.restype = ctypes.c_uint64
 
 
 class QloraError(RuntimeError):
@@ -108,6 +111,11 @@ def _ptr(t):
 
 def qlora_version():
     return int(lib.qlora_version())
+
+
+def qlora_launch_count():
+    """Kernels launched by the library in this process so far."""
+    return int(lib.qlora_launch_count())
 
 
 def qlora_status_string(status):

@@ -1,6 +1,6 @@
 """Build ``libqlora.so`` in-tree with nvcc for sm_100a.
 
-    python -m bit_nf4_quantized_06_b200.build [--force] [-v]
+    python bit_nf4_quantized_06_b200/build.py [--force] [-v] [--ptxas-info]
 
 Each ``csrc/*.cu`` is compiled separately (in parallel) with
 ``-gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`` and linked into a

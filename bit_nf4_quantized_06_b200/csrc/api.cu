@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include <cudaTypedefs.h>
@@ -73,6 +74,7 @@ struct DevState {
   bool ok = false;
   int sms = 148;
   bool attrs = false;
+  int pair_clusters = 0;   // CTA pairs of k_tc_pair that can be resident at once
 };
 std::mutex g_mu;
 DevState g_dev[64];
@@ -103,7 +105,39 @@ cudaError_t set_small_attrs() {
   return set_tc_attr<BN, A_TMA_MN, B_TMA_MN, EPI_F32_ROWS>();
 }
 
-qlora_status_t device_ready(int* sms_out) {
+template <int AS, int NH>
+cudaError_t pair_clusters_of(int* out) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(448, 1, 1);
+  cfg.dynamicSmemBytes = tc_pair_smem_bytes(NH);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaFuncSetAttribute(k_tc_pair<AS, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       tc_pair_smem_bytes(NH));
+  if (e != cudaSuccess) return e;
+  return cudaOccupancyMaxActiveClusters(out, k_tc_pair<AS, NH>, &cfg);
+}
+
+// How many 2-CTA clusters of the pair kernels fit on the device at once (one
+// CTA per SM, clusters confined to a GPC); also sets their shared-memory limit.
+cudaError_t pair_clusters(int* out) {
+  int n[4] = {0, 0, 0, 0};
+  cudaError_t e;
+  if ((e = pair_clusters_of<A_DQ_K, 1>(&n[0])) != cudaSuccess) return e;
+  if ((e = pair_clusters_of<A_DQ_K, 2>(&n[1])) != cudaSuccess) return e;
+  if ((e = pair_clusters_of<A_DQ_MN, 1>(&n[2])) != cudaSuccess) return e;
+  if ((e = pair_clusters_of<A_DQ_MN, 2>(&n[3])) != cudaSuccess) return e;
+  *out = std::min(std::min(n[0], n[1]), std::min(n[2], n[3]));
+  return (*out > 0) ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+qlora_status_t device_ready(int* sms_out, int* pairs_out = nullptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
@@ -117,8 +151,7 @@ qlora_status_t device_ready(int* sms_out) {
   }
   if (!st.ok) return QLORA_ERR_UNSUPPORTED_DEVICE;
   if (!st.attrs) {
-    cudaError_t e = set_tc_attr<256, A_DQ_K, B_TMA_K, EPI_BF16_T>();
-    if (e == cudaSuccess) e = set_tc_attr<256, A_DQ_MN, B_TMA_K, EPI_BF16_T>();
+    cudaError_t e = pair_clusters(&st.pair_clusters);
     if (e == cudaSuccess) e = set_small_attrs<64>();
     if (e == cudaSuccess) e = set_small_attrs<128>();
     if (e == cudaSuccess) e = set_small_attrs<192>();
@@ -127,6 +160,7 @@ qlora_status_t device_ready(int* sms_out) {
     st.attrs = true;
   }
   if (sms_out) *sms_out = st.sms;
+  if (pairs_out) *pairs_out = st.pair_clusters;
   return QLORA_OK;
 }
 
@@ -158,7 +192,7 @@ bool map_bf16(CUtensorMap* m, const void* ptr, int64_t outer, int64_t inner, int
 
 // Split count for a reduction of `ktiles` 64-wide tiles over `tiles` output tiles.
 int pick_splits(int64_t tiles, int64_t ktiles, int sms) {
-  int64_t s = cdiv(sms, std::max<int64_t>(1, tiles));
+  int64_t s = sms / std::max<int64_t>(1, tiles);
   s = std::min<int64_t>(s, ktiles);
   s = std::min<int64_t>(s, 16);
   s = std::max<int64_t>(s, 1);
@@ -212,7 +246,11 @@ qlora_status_t check_nf4(const qlora_nf4_t* q) {
   return QLORA_OK;
 }
 
+std::atomic<uint64_t> g_launches{0};
+
+// Every kernel launch is followed by this check; it also counts the launch.
 inline qlora_status_t launch_status() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
@@ -222,22 +260,69 @@ CUtensorMap zero_map() {
   return m;
 }
 
+// Persistent launch: one CTA per SM at most, each walking the tile list.
 template <int BN, int AS, int BS, int EP>
-qlora_status_t launch_tc(dim3 grid, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& b,
+qlora_status_t launch_tc(int sms, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& b,
                          const CUtensorMap& bl, const CUtensorMap& c, const TcParams& p) {
-  k_tc_gemm<BN, AS, BS, EP, 4><<<grid, 192, tc_smem_bytes<BN, AS, BS, 4>(), st>>>(a, b, bl, c, p);
+  const int64_t tiles = static_cast<int64_t>(p.tiles_rows) * p.tiles_cols * p.splits;
+  if (tiles <= 0) return QLORA_ERR_SHAPE;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, sms));
+  k_tc_gemm<BN, AS, BS, EP, 4><<<grid, tc_threads<AS>(), tc_smem_bytes<BN, AS, BS, 4>(), st>>>(a, b, bl, c, p);
   return launch_status();
 }
 
+// Persistent CTA-pair launch: at most `pairs` clusters of two CTAs.
+template <int AS, int NH>
+qlora_status_t launch_pair_nh(int pairs, cudaStream_t st, const CUtensorMap& b, const CUtensorMap& bl,
+                              const CUtensorMap& c, const TcParams& p) {
+  const int64_t tiles = static_cast<int64_t>(p.tiles_rows) * p.tiles_cols;
+  if (tiles <= 0 || pairs <= 0) return QLORA_ERR_SHAPE;
+  const unsigned nclusters = static_cast<unsigned>(std::min<int64_t>(tiles, pairs));
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * nclusters, 1, 1);
+  cfg.blockDim = dim3(448, 1, 1);
+  cfg.dynamicSmemBytes = tc_pair_smem_bytes(NH);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc_pair<AS, NH>, b, bl, c, p);
+  if (e != cudaSuccess) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+// Token groups of 256 per restored weight tile: two once there are more than
+// 256 tokens (each restored tile then feeds 512 tokens), else one.
+inline int pair_nh(int64_t m) { return m > 256 ? 2 : 1; }
+
+template <int AS>
+qlora_status_t launch_pair(int pairs, int64_t m, cudaStream_t st, const CUtensorMap& b, const CUtensorMap& bl,
+                           const CUtensorMap& c, TcParams p) {
+  if (pair_nh(m) == 2) {
+    p.tiles_cols = static_cast<int32_t>(cdiv(m, 512));
+    return launch_pair_nh<AS, 2>(pairs, st, b, bl, c, p);
+  }
+  p.tiles_cols = static_cast<int32_t>(cdiv(m, 256));
+  return launch_pair_nh<AS, 1>(pairs, st, b, bl, c, p);
+}
+
 template <int AS, int BS>
-qlora_status_t launch_small(int32_t r64, dim3 grid, cudaStream_t st, const CUtensorMap& a,
+qlora_status_t launch_small(int32_t r64, int sms, cudaStream_t st, const CUtensorMap& a,
                             const CUtensorMap& b, const TcParams& p) {
   const CUtensorMap z = zero_map();
   switch (r64) {
-    case 64: return launch_tc<64, AS, BS, EPI_F32_ROWS>(grid, st, a, b, z, z, p);
-    case 128: return launch_tc<128, AS, BS, EPI_F32_ROWS>(grid, st, a, b, z, z, p);
-    case 192: return launch_tc<192, AS, BS, EPI_F32_ROWS>(grid, st, a, b, z, z, p);
-    case 256: return launch_tc<256, AS, BS, EPI_F32_ROWS>(grid, st, a, b, z, z, p);
+    case 64: return launch_tc<64, AS, BS, EPI_F32_ROWS>(sms, st, a, b, z, z, p);
+    case 128: return launch_tc<128, AS, BS, EPI_F32_ROWS>(sms, st, a, b, z, z, p);
+    case 192: return launch_tc<192, AS, BS, EPI_F32_ROWS>(sms, st, a, b, z, z, p);
+    case 256: return launch_tc<256, AS, BS, EPI_F32_ROWS>(sms, st, a, b, z, z, p);
     default: return QLORA_ERR_SHAPE;
   }
 }
@@ -264,11 +349,13 @@ qlora_status_t lora_product(const CUtensorMap& ma, const CUtensorMap& mb, int64_
   p.kt_main = static_cast<int32_t>(cdiv(kdim, 64));
   p.kt_lora = 0;
   p.kt_split = sp.kt_split;
+  p.tiles_rows = static_cast<int32_t>(cdiv(rows, 128));
+  p.tiles_cols = 1;
+  p.splits = sp.splits;
   p.out = part;
   p.ldo = r64;
   p.rows_pad = static_cast<int32_t>(sp.rows_pad);
-  const dim3 grid(static_cast<unsigned>(cdiv(rows, 128)), 1, static_cast<unsigned>(sp.splits));
-  qlora_status_t s = launch_small<AS, BS>(r64, grid, st, ma, mb, p);
+  qlora_status_t s = launch_small<AS, BS>(r64, sms, st, ma, mb, p);
   if (s != QLORA_OK) return s;
   ReduceParams rp{};
   rp.part = part;
@@ -314,6 +401,8 @@ using namespace qlora;
 extern "C" {
 
 int32_t qlora_version(void) { return 100; }
+
+uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* qlora_status_string(qlora_status_t s) {
   switch (s) {
@@ -398,11 +487,11 @@ qlora_status_t qlora_dequantize(const qlora_nf4_t* q, void* w_bf16_out, void* st
 qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t m, const void* a,
                                    const void* b, int32_t r, float alpha, void* y, void* u_out,
                                    void* ws, size_t ws_bytes, int32_t path, void* stream) {
-  int sms = 0;
+  int sms = 0, pairs = 0;
   qlora_status_t s = check_nf4(q);
   if (s != QLORA_OK) return s;
   if (path < QLORA_FWD_AUTO || path > QLORA_FWD_GEMV) return QLORA_ERR_INVALID_ARG;
-  if ((s = device_ready(&sms)) != QLORA_OK) return s;
+  if ((s = device_ready(&sms, &pairs)) != QLORA_OK) return s;
   const LinearArgs la{q, m, r, alpha, ws, ws_bytes};
   if ((s = check_linear(la, sms)) != QLORA_OK) return s;
   if (m == 0) return QLORA_OK;
@@ -479,7 +568,7 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
   if (s != QLORA_OK) return s;
 
   // y^T tiles: A = restored W (on chip), B = x, plus u' B^T as extra k-tiles
-  if (!map_bf16(&m_x_b, xb, m, k, k, 256) || !map_bf16(&m_u, u_pad, m, r64, r64, 256) ||
+  if (!map_bf16(&m_x_b, xb, m, k, k, 128) || !map_bf16(&m_u, u_pad, m, r64, r64, 128) ||
       !map2d(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->codes, static_cast<uint64_t>(k / 2),
              static_cast<uint64_t>(n), static_cast<uint64_t>(k / 2), 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
     return QLORA_ERR_CUDA;
@@ -489,9 +578,13 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
   p.kt_main = static_cast<int32_t>(k / 64);
   p.kt_lora = r64 / 64;
   p.kt_split = p.kt_main;
+  p.tiles_rows = static_cast<int32_t>(cdiv(n, 256));
+  p.tiles_cols = static_cast<int32_t>(cdiv(m, 256));
+  p.splits = 1;
   p.q2 = q->scale_codes;
   p.smax = q->absmax;
   p.kblocks = k / 64;
+  p.nblocks = n * (k / 64);
   p.w_rows = n;
   p.w_cols = k;
   std::memcpy(p.cb, tables().cb, sizeof(p.cb));
@@ -500,9 +593,7 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
   p.lora_r = (r % 8 != 0) ? r64 : r;
   p.out = y;
   p.ldo = n;
-  const dim3 grid(static_cast<unsigned>(cdiv(n, 128)), static_cast<unsigned>(cdiv(m, 256)), 1);
-  const CUtensorMap z = zero_map();
-  return launch_tc<256, A_DQ_K, B_TMA_K, EPI_BF16_T>(grid, st, z, m_x_b, m_u, m_codes, p);
+  return launch_pair<A_DQ_K>(pairs, m, st, m_x_b, m_u, m_codes, p);
 }
 
 qlora_status_t qlora_linear_fwd(const qlora_nf4_t* q, const void* x, int64_t m, const void* a, const void* b,
@@ -514,10 +605,10 @@ qlora_status_t qlora_linear_fwd(const qlora_nf4_t* q, const void* x, int64_t m, 
 qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void* u, const void* dy, int64_t m,
                                 const void* a, const void* b, int32_t r, float alpha, void* dx, float* da,
                                 float* db, void* ws, size_t ws_bytes, void* stream) {
-  int sms = 0;
+  int sms = 0, pairs = 0;
   qlora_status_t s = check_nf4(q);
   if (s != QLORA_OK) return s;
-  if ((s = device_ready(&sms)) != QLORA_OK) return s;
+  if ((s = device_ready(&sms, &pairs)) != QLORA_OK) return s;
   const LinearArgs la{q, m, r, alpha, ws, ws_bytes};
   if ((s = check_linear(la, sms)) != QLORA_OK) return s;
   if (x == nullptr || dy == nullptr || a == nullptr || b == nullptr || da == nullptr || db == nullptr)
@@ -590,7 +681,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
   // plus v' A_lora as extra k-tiles
   if (dx != nullptr) {
     CUtensorMap m_dy_b, m_v, m_codes;
-    if (!map_bf16(&m_dy_b, dyb, m, n, n, 256) || !map_bf16(&m_v, v_pad, m, r64, r64, 256) ||
+    if (!map_bf16(&m_dy_b, dyb, m, n, n, 128) || !map_bf16(&m_v, v_pad, m, r64, r64, 128) ||
         !map2d(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->codes, static_cast<uint64_t>(k / 2),
                static_cast<uint64_t>(n), static_cast<uint64_t>(k / 2), 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
       return QLORA_ERR_CUDA;
@@ -600,9 +691,13 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
     p.kt_main = static_cast<int32_t>(cdiv(n, 64));
     p.kt_lora = r64 / 64;
     p.kt_split = p.kt_main;
+    p.tiles_rows = static_cast<int32_t>(cdiv(k, 256));
+    p.tiles_cols = static_cast<int32_t>(cdiv(m, 256));
+    p.splits = 1;
     p.q2 = q->scale_codes;
     p.smax = q->absmax;
     p.kblocks = k / 64;
+    p.nblocks = n * (k / 64);
     p.w_rows = n;
     p.w_cols = k;
     std::memcpy(p.cb, tables().cb, sizeof(p.cb));
@@ -611,9 +706,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
     p.lora_r = r;
     p.out = dx;
     p.ldo = k;
-    const dim3 grid(static_cast<unsigned>(cdiv(k, 128)), static_cast<unsigned>(cdiv(m, 256)), 1);
-    const CUtensorMap z = zero_map();
-    s = launch_tc<256, A_DQ_MN, B_TMA_K, EPI_BF16_T>(grid, st, z, m_dy_b, m_v, m_codes, p);
+    s = launch_pair<A_DQ_MN>(pairs, m, st, m_dy_b, m_v, m_codes, p);
     if (s != QLORA_OK) return s;
   }
 

@@ -68,11 +68,15 @@ struct TcParams {
   int32_t cols;         // extent of the D columns
   int32_t kt_main;      // main k-tiles (64 each) in the reduction
   int32_t kt_lora;      // extra k-tiles appended after the main ones (LoRA term)
-  int32_t kt_split;     // main k-tiles per split (gridDim.z splits)
+  int32_t kt_split;     // main k-tiles per split
+  int32_t tiles_rows;   // 128-row tiles
+  int32_t tiles_cols;   // BN-column tiles
+  int32_t splits;       // reduction splits (tile index = (row tile * tiles_cols + col tile) * splits + split)
   // restored-weight operand (A_DQ_*)
   const uint8_t* q2;
   const float* smax;
   int64_t kblocks;      // K/64 of the weight: blocks per weight row
+  int64_t nblocks;      // N*K/64: length of q2
   int64_t w_rows;       // N of the weight (rows of W)
   int64_t w_cols;       // K of the weight
   float cb[16];
@@ -86,15 +90,41 @@ struct TcParams {
   int32_t rows_pad;     // EPI_F32_ROWS: rows per split slab
 };
 
+// Persistent kernel: gridDim.x CTAs (at most one per SM) walk the tiles
+// blockIdx.x, blockIdx.x + gridDim.x, ...
 template <int BN, int AS, int BS, int EP, int STAGES>
 __global__ void k_tc_gemm(const __grid_constant__ CUtensorMap tm_a,
                           const __grid_constant__ CUtensorMap tm_b,
                           const __grid_constant__ CUtensorMap tm_b_lora,
                           const __grid_constant__ CUtensorMap tm_codes, TcParams p);
 
+constexpr int kScalePrefetch = 4;  // k-tiles of scale codes fetched ahead by each A-producer thread
+
+template <int AS>
+constexpr bool tc_dq() { return AS == A_DQ_K || AS == A_DQ_MN; }
+
+template <int AS>
+constexpr int tc_threads() { return tc_dq<AS>() ? 448 : 192; }
+
 template <int BN, int AS, int BS, int STAGES>
 constexpr int tc_smem_bytes() {
-  return STAGES * (16384 + BN * 128 + ((AS == A_DQ_K || AS == A_DQ_MN) ? 4096 : 0)) + 1024 + 256;
+  return STAGES * (16384 + BN * 128 + (tc_dq<AS>() ? 4096 : 0)) + 1024 + 256 +
+         (tc_dq<AS>() ? 2 * kScalePrefetch * 128 * 8 : 0);
+}
+
+// CTA-pair (cta_group::2) fused restore + GEMM for the forward (A_DQ_K) and
+// dX (A_DQ_MN): clusters of two CTAs walk 256 x (256 NH) tiles; tiles_rows
+// counts 256-row tiles and tiles_cols (256 NH)-column tiles. Launched with
+// cluster dimension 2.
+// NH = token groups of 256 per restored A tile (1 or 2).
+constexpr int pair_stages(int nh) { return nh == 1 ? 6 : 4; }
+
+template <int AS, int NH>
+__global__ void k_tc_pair(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b_lora,
+                          const __grid_constant__ CUtensorMap tm_codes, TcParams p);
+
+constexpr int tc_pair_smem_bytes(int nh) {
+  return pair_stages(nh) * (16384 + nh * 16384 + 4096) + 1024 + 256 + 2 * kScalePrefetch * 128 * 8;
 }
 
 // Split reductions (fixed order over splits -> deterministic).

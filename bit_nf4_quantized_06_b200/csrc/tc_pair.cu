@@ -1,0 +1,442 @@
+// Fused NF4-restore + tcgen05 GEMM on CTA pairs (cta_group::2), sm_100a.
+//
+// A cluster of two CTAs computes a (256 NH) tokens x 256 features tile of the
+// output (y for the forward, dX for the backward), accumulating in fp32 in
+// tensor memory with tokens on the tensor-memory lanes:
+//
+//   D_h[256 tokens x 256 features] += T_h[256 x 64] * W[256 x 64]^T   per k-tile, h < NH
+//
+// T_h is a 256-token slice of the input (x or dY), loaded by TMA, 128 tokens
+// per CTA. W is the 256-feature slice of the restored weight: CTA r restores
+// features [128 r, 128 r + 128) from the packed codes into the 128-byte
+// swizzled layout the tensor core reads (K-major for the forward, MN-major
+// for dX, whose reduction runs along d_out while the 4-bit blocks run along
+// d_in). The even CTA issues the pair MMAs, which read both CTAs' shared
+// memory; each restored W tile serves 256 NH tokens. The LoRA term is appended
+// as extra k-tiles of the same accumulators: T = u' (or v') from TMA and
+// W = B_lora rows (or A_lora rows) copied by the restore warps.
+// ("48GB GPU Fine-Tuning a 65B Model ...", § "QLoRA Puts the Two Methods in
+// Different Places": each block of W is restored to bf16 before it meets the
+// input, and gradients reach x through the restored W; W gets none.)
+//
+// With tokens on the lanes, each epilogue thread owns one output row and
+// writes 64 contiguous bytes per 32 accumulator columns (16-byte stores).
+// NH = 2 uses the whole tensor memory for one tile (its drain does not
+// overlap the next tile); NH = 1 keeps two accumulators and overlaps it.
+//
+// Warp roles in each CTA (448 threads):
+//   warp 0      TMA: this CTA's token slices (completion counted on the even
+//               CTA's barrier) and this CTA's code tile (local barrier)
+//   warp 1      tensor-memory allocation for the pair; in the even CTA one
+//               lane issues the pair MMAs and commits to both CTAs' barriers
+//   warps 2-9   restore: two groups of four warps take alternate k-tiles
+//   warps 10-13 epilogue: drain this CTA's 128 token rows
+//
+// Every wait is bounded; every TMA load fills only the issuing CTA's shared
+// memory; the MMA's completion reaches the odd CTA through a commit to its
+// barrier's cluster address.
+#include "kernels.h"
+#include "nf4_dev.cuh"
+#include "ptx.cuh"
+#include "tc_common.cuh"
+
+namespace qlora {
+
+using namespace tcd;
+
+template <int AS, int NH>
+__global__ void __launch_bounds__(448, 1)
+    k_tc_pair(const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_t_lora,
+              const __grid_constant__ CUtensorMap tm_codes, TcParams p) {
+  constexpr int STAGES = pair_stages(NH);
+  constexpr bool W_MN = (AS == A_DQ_MN);
+  constexpr uint32_t W_BYTES = 16384;        // 128 features x 64 k, bf16 (restored here)
+  constexpr uint32_t T_HALF = 16384;         // 128 tokens x 64 k, bf16 (this CTA's share of one MMA)
+  constexpr uint32_t T_BYTES = NH * T_HALF;
+  constexpr uint32_t C_BYTES = 4096;         // packed codes for the 128 features
+  constexpr uint32_t STAGE_BYTES = W_BYTES + T_BYTES + C_BYTES;
+  constexpr uint32_t IDESC = idesc_bf16_f32(256, 256, false, W_MN);
+  constexpr uint32_t TILE_COLS = 256 * NH;   // accumulator columns per tile
+  constexpr int NBUF = (NH == 1) ? 2 : 1;    // accumulator buffers (double-buffered when they fit)
+  constexpr uint32_t TMEM_ALLOC = 512;
+  constexpr int PD = kScalePrefetch;
+  static_assert(NBUF * TILE_COLS <= TMEM_ALLOC, "tensor memory");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const ctl = smem_raw + (base - raw) + STAGES * STAGE_BYTES;
+  const uint32_t bar0 = base + STAGES * STAGE_BYTES;
+  auto bar_full = [&](int s) { return bar0 + 8u * s; };                 // even CTA: token slices of both
+  auto bar_codes = [&](int s) { return bar0 + 8u * (STAGES + s); };     // local code tile
+  auto bar_wfull = [&](int s) { return bar0 + 8u * (2 * STAGES + s); }; // even CTA: 8 restore warps
+  auto bar_empty = [&](int s) { return bar0 + 8u * (3 * STAGES + s); }; // local, from the MMA
+  auto bar_accf = [&](int b) { return bar0 + 8u * (4 * STAGES + b); };  // local, from the MMA
+  auto bar_acce = [&](int b) { return bar0 + 8u * (4 * STAGES + 2 + b); };  // even CTA: 8 epilogue warps
+  const uint32_t bar_fin = bar0 + 8u * (4 * STAGES + 4);
+  uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(ctl + 8 * (4 * STAGES + 5));
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(ctl + 8 * (4 * STAGES + 5) + 4);
+  const uint32_t ring = bar0 + 256;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int ntile_total = p.tiles_rows * p.tiles_cols;  // 256-feature x (256 NH)-token tiles
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_codes(s), 1);
+      mbar_init(bar_wfull(s), 8);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf(b), 1);
+      mbar_init(bar_acce(b), 8);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_holder), TMEM_ALLOC);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();   // barriers initialised and tensor memory allocated in both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  // tile -> first feature of this CTA's restored slice, first token of the tile
+  auto tile_feat = [&](int tile) { return (tile / p.tiles_cols) * 256 + 128 * static_cast<int>(rank); };
+  auto tile_tok = [&](int tile) { return (tile % p.tiles_cols) * static_cast<int>(TILE_COLS); };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_t);
+      tma_prefetch_desc(&tm_codes);
+      if (p.kt_lora > 0) tma_prefetch_desc(&tm_t_lora);
+      const int ntiles = p.kt_main + p.kt_lora;
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < ntile_total; tile += npairs) {
+        const int f0 = tile_feat(tile);
+        const int tok = tile_tok(tile) + 128 * static_cast<int>(rank);
+        for (int t = 0; t < ntiles; ++t, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(bar_empty(s), ph ^ 1, abort_flag, QLORA_DEV_TIMEOUT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          const uint32_t w_s = base + s * STAGE_BYTES;
+          const uint32_t t_s = w_s + W_BYTES;
+          const uint32_t c_s = t_s + T_BYTES;
+          const uint32_t full_even = mapa_shared(bar_full(s), 0);
+          if (leader) mbar_arrive_expect_tx(bar_full(s), 2 * T_BYTES);
+          if (t < p.kt_main) {
+#pragma unroll
+            for (int h = 0; h < NH; ++h) tma_load_2d_pair(t_s + h * T_HALF, &tm_t, full_even, t * 64, tok + 256 * h);
+            mbar_arrive_expect_tx(bar_codes(s), C_BYTES);
+            if (AS == A_DQ_K)
+              tma_load_2d(c_s, &tm_codes, bar_codes(s), t * 32, f0);
+            else
+              tma_load_2d(c_s, &tm_codes, bar_codes(s), f0 / 2, t * 64);
+          } else {
+#pragma unroll
+            for (int h = 0; h < NH; ++h)
+              tma_load_2d_pair(t_s + h * T_HALF, &tm_t_lora, full_even, (t - p.kt_main) * 64, tok + 256 * h);
+            mbar_arrive(bar_codes(s));  // keeps the code barrier's phase in step
+          }
+        }
+      }
+      // the loads this thread started have landed once the MMA released their stage
+      for (int j = max(0, it - STAGES); j < it; ++j) {
+        drain_wait(bar_empty(j % STAGES), (j / STAGES) & 1);
+        drain_wait(bar_codes(j % STAGES), (j / STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer (even CTA)
+    if (leader && lane == 0) {
+      const int ntiles = p.kt_main + p.kt_lora;
+      int it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < ntile_total; tile += npairs, ++tcount) {
+        const int b = tcount % NBUF;
+        const uint32_t aph = (tcount / NBUF) & 1;
+        if (!mbar_wait(bar_acce(b), aph ^ 1, abort_flag, QLORA_DEV_TIMEOUT_MMA)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + b * TILE_COLS;
+        for (int t = 0; t < ntiles; ++t, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(bar_full(s), ph, abort_flag, QLORA_DEV_TIMEOUT_MMA) ||
+              !mbar_wait(bar_wfull(s), ph, abort_flag, QLORA_DEV_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t w_s = base + s * STAGE_BYTES;
+          const uint32_t t_s = w_s + W_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t dw = W_MN ? smem_desc_sw128(w_s + kk * 2048, 8192, 1024)
+                                     : smem_desc_sw128(w_s + kk * 32, 16, 1024);
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+              const uint64_t dt = smem_desc_sw128(t_s + h * T_HALF + kk * 32, 16, 1024);
+              tc_mma_pair(d_tmem + h * 256, dt, dw, IDESC, (t > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit_pair(bar_empty(s));
+          tc_commit_pair(mapa_shared(bar_empty(s), 1));
+        }
+        if (ok) {
+          tc_commit_pair(bar_accf(b));
+          tc_commit_pair(mapa_shared(bar_accf(b), 1));
+        }
+      }
+      tc_commit_pair(bar_fin);
+      drain_wait(bar_fin, 0);
+    }
+  } else if (warp < 10) {
+    // ---------------------------------------------------------------- restore
+    const int grp = (warp - 2) >> 2;                 // 0: warps 2-5, 1: warps 6-9
+    const int tid = threadIdx.x - 64 - 128 * grp;    // 0..127
+    const int ipt = p.kt_main + p.kt_lora;
+    const int my_tiles = (ntile_total - pair + npairs - 1) / npairs;
+    const int items = my_tiles * ipt;
+    const uint32_t slot0 = ring + grp * (PD * 128 * 8) + tid * 8;
+
+    // cursor over this group's items j = grp, grp + 2, ...: k-tile t of a
+    // tile whose restored slice starts at feature f0
+    struct Cursor {
+      int j, t, tile, f0;
+    };
+    auto advance = [&](Cursor& c) {
+      c.j += 2;
+      c.t += 2;
+      while (c.t >= ipt) {
+        c.t -= ipt;
+        c.tile += npairs;
+        c.f0 = tile_feat(c.tile);
+      }
+    };
+    // this thread's weight block for k-tile t (-1 = padding)
+    auto block_of = [&](int f0, int t) -> int64_t {
+      if (AS == A_DQ_K) {
+        const int64_t n = f0 + tid;
+        return (n < p.w_rows) ? n * p.kblocks + t : -1;
+      } else {
+        const int64_t n = static_cast<int64_t>(t) * 64 + (tid >> 1);
+        const int64_t kcol = f0 + 64 * (tid & 1);
+        return (n < p.w_rows && kcol < p.w_cols) ? n * p.kblocks + (kcol >> 6) : -1;
+      }
+    };
+    auto issue = [&](const Cursor& c, int k) {
+      if (c.j < items && c.t < p.kt_main) {
+        const int64_t bi = block_of(c.f0, c.t);
+        const uint32_t slot = slot0 + k * (128 * 8);
+        if (bi >= 0) {
+          const int64_t w4 = bi & ~int64_t(3);
+          const int64_t left = p.nblocks - w4;
+          cp_async4(slot, p.q2 + w4, static_cast<uint32_t>(left < 4 ? left : 4));
+          cp_async4(slot + 4, p.smax + (bi >> 8), 4);
+        } else {
+          cp_async4(slot, p.q2, 0);
+          cp_async4(slot + 4, p.smax, 0);
+        }
+      }
+      cp_async_commit();
+    };
+
+    Cursor cur{grp, grp, pair, 0};
+    cur.f0 = tile_feat(cur.tile);
+    while (cur.t >= ipt) {
+      cur.t -= ipt;
+      cur.tile += npairs;
+      cur.f0 = tile_feat(cur.tile);
+    }
+    Cursor pre = cur;
+#pragma unroll 1
+    for (int k = 0; k < PD - 1; ++k) {
+      issue(pre, k);
+      advance(pre);
+    }
+    int slot_use = 0, slot_issue = PD - 1;
+    const uint32_t wfull_even0 = mapa_shared(bar_wfull(0), 0);
+
+#pragma unroll 1
+    for (; cur.j < items; advance(cur)) {
+      issue(pre, slot_issue);
+      advance(pre);
+      slot_issue = (slot_issue + 1 == PD) ? 0 : slot_issue + 1;
+      const int j = cur.j;
+      const int s = j % STAGES;
+      const uint32_t ph = (j / STAGES) & 1;
+      const int t = cur.t;
+      const int f0 = cur.f0;
+      const uint32_t w_s = base + s * STAGE_BYTES;
+      const uint32_t c_s = w_s + W_BYTES + T_BYTES;
+      bool ok = mbar_wait(bar_empty(s), ph ^ 1, abort_flag, QLORA_DEV_TIMEOUT_APROD);
+      if (!warp_all(ok)) break;
+      if (t < p.kt_main) {
+        cp_async_wait<PD - 1>();
+        const int64_t bi = block_of(f0, t);
+        const uint32_t slot = slot0 + slot_use * (128 * 8);
+        float sh = 0.0f;
+        if (bi >= 0) {
+          const uint32_t qw = lds32(slot);
+          const uint32_t q2 = (qw >> (8 * static_cast<uint32_t>(bi & 3))) & 0xFFu;
+          sh = restored_scale(q2, __uint_as_float(lds32(slot + 4)));
+        }
+        const Nf4Table tb = make_table(p.cb, sh);
+        ok = mbar_wait(bar_codes(s), ph, abort_flag, QLORA_DEV_TIMEOUT_APROD);
+        if (!warp_all(ok)) break;
+        uint32_t src, dst, sw;
+        if (AS == A_DQ_K) {
+          src = c_s + tid * 32;
+          dst = w_s + tid * 128;
+          sw = tid & 7;
+        } else {
+          const int nr = tid >> 1;
+          src = c_s + nr * 64 + (tid & 1) * 32;
+          dst = w_s + (tid & 1) * 8192 + nr * 128;
+          sw = nr & 7;
+        }
+        const uint4 c0 = lds128(src);
+        const uint4 c1 = lds128(src + 16);
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          uint32_t o[4];
+          lookup8(tb, words[w], o);
+          sts128(dst + ((w ^ sw) << 4), o[0], o[1], o[2], o[3]);
+        }
+      } else {
+        const int lt = t - p.kt_main;
+        if (AS == A_DQ_K) {
+          // forward: rows of B_lora (one output feature per thread), 64 ranks
+          const int64_t n = f0 + tid;
+          const uint32_t dst = w_s + tid * 128;
+          const uint32_t sw = tid & 7;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 v = make_uint4(0, 0, 0, 0);
+            const int jj = lt * 64 + 8 * c;
+            if (n < p.w_rows && jj < p.lora_r)
+              v = __ldg(reinterpret_cast<const uint4*>(p.lora + n * p.lora_ld + jj));
+            sts128(dst + ((c ^ sw) << 4), v.x, v.y, v.z, v.w);
+          }
+        } else {
+          // dX: rows of A_lora (rank = reduction index), 64 of its d_in columns
+          const int nr = tid >> 1;
+          const int jr = lt * 64 + nr;
+          const int64_t kcol = f0 + 64 * (tid & 1);
+          const bool valid = kcol < p.w_cols && jr < p.lora_r;
+          const uint32_t dst = w_s + (tid & 1) * 8192 + nr * 128;
+          const uint32_t sw = nr & 7;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (valid) v = __ldg(reinterpret_cast<const uint4*>(p.lora + jr * p.lora_ld + kcol + 8 * c));
+            sts128(dst + ((c ^ sw) << 4), v.x, v.y, v.z, v.w);
+          }
+        }
+      }
+      slot_use = (slot_use + 1 == PD) ? 0 : slot_use + 1;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(bar_wfull(s));
+        else
+          mbar_arrive_cluster(wfull_even0 + 8u * s);
+      }
+    }
+    cp_async_wait<0>();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // TMEM lanes [32 q, 32 q + 32) belong to warp % 4
+    const uint32_t acce_even0 = mapa_shared(bar_acce(0), 0);
+    const bool vec_ok = (p.ldo % 8) == 0;
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+    int tcount = 0;
+    for (int tile = pair; tile < ntile_total; tile += npairs, ++tcount) {
+      const int b = tcount % NBUF;
+      const uint32_t aph = (tcount / NBUF) & 1;
+      bool ok = mbar_wait(bar_accf(b), aph, abort_flag, QLORA_DEV_TIMEOUT_EPI);
+      if (!warp_all(ok)) break;
+      tc_fence_after();
+      const int f0 = (tile / p.tiles_cols) * 256;   // first feature of the pair's tile
+      const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+#pragma unroll 1
+      for (int h = 0; h < NH; ++h) {
+        const int token = tile_tok(tile) + 256 * h + 128 * static_cast<int>(rank) + quarter * 32 + lane;
+        __nv_bfloat16* orow = out + static_cast<int64_t>(token) * p.ldo;
+        const uint32_t taddr = tmem_base + b * TILE_COLS + h * 256 + lane_base;
+#pragma unroll 1
+        for (int ch = 0; ch < 8; ch += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(taddr + ch * 32, r0);
+          tmem_ld_32x32b_x32(taddr + ch * 32 + 32, r1);
+          tc_wait_ld();
+          if (token < p.cols) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              const uint32_t* r = half ? r1 : r0;
+              const int fc = f0 + (ch + half) * 32;
+              if (vec_ok && fc + 32 <= p.rows) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + fc);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                  dst[v] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
+                                      pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
+                                      pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
+                                      pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+                }
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  if (fc + i < p.rows) orow[fc + i] = __float2bfloat16_rn(__uint_as_float(r[i]));
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(bar_acce(b));
+        else
+          mbar_arrive_cluster(acce_even0 + 8u * b);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();   // no CTA leaves while its pair still reads its shared or tensor memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_ALLOC);
+  }
+}
+
+#define QLORA_PAIR_INST(AS, NH)                                                                         \
+  template __global__ void k_tc_pair<AS, NH>(const __grid_constant__ CUtensorMap,                       \
+                                             const __grid_constant__ CUtensorMap,                       \
+                                             const __grid_constant__ CUtensorMap, TcParams);
+QLORA_PAIR_INST(A_DQ_K, 1)
+QLORA_PAIR_INST(A_DQ_K, 2)
+QLORA_PAIR_INST(A_DQ_MN, 1)
+QLORA_PAIR_INST(A_DQ_MN, 2)
+
+}  // namespace qlora

@@ -150,6 +150,11 @@ QLORA_API qlora_status_t qlora_device_status(void *stream, uint32_t *bits);
 /* Static description of a status code. */
 QLORA_API const char *qlora_status_string(qlora_status_t s);
 
+/* Number of kernels this library has launched in this process (all devices,
+ * all streams) since it was loaded. Host only; lets a caller count the
+ * device work behind a sequence of calls. */
+QLORA_API uint64_t qlora_launch_count(void);
+
 /* Library version as major*10000 + minor*100 + patch. */
 QLORA_API int32_t qlora_version(void);
 
