@@ -10,7 +10,7 @@ Functions carry the C names:
 
     qlora_nf4_bytes, qlora_nf4_codebook, qlora_quantize_nf4, qlora_dequantize,
     qlora_workspace_bytes, qlora_linear_fwd, qlora_linear_fwd_ex,
-    qlora_linear_bwd, qlora_device_status, qlora_status_string, qlora_version,
+    qlora_linear_fwd_noalloc, qlora_linear_bwd, qlora_device_status, qlora_status_string, qlora_version,
     qlora_launch_count
 """
 
@@ -20,7 +20,8 @@ import os
 __all__ = [
     "LIB_PATH", "lib", "QloraError", "NF4Weight", "Nf4Struct",
     "qlora_nf4_bytes", "qlora_nf4_codebook", "qlora_quantize_nf4", "qlora_dequantize",
-    "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_fwd_ex", "qlora_linear_bwd",
+    "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_fwd_ex", "qlora_linear_fwd_noalloc",
+    "qlora_linear_bwd",
     "qlora_device_status", "qlora_status_string", "qlora_version", "qlora_launch_count",
     "FWD_AUTO", "FWD_GEMM", "FWD_GEMV",
 ]
@@ -68,6 +69,8 @@ lib.qlora_linear_fwd.restype = ctypes.c_int
 lib.qlora_linear_fwd_ex.argtypes = [_P(Nf4Struct), _vp, _i64, _vp, _vp, _i32, _f32, _vp, _vp, _vp, _sz, _i32,
                                     _vp]
 lib.qlora_linear_fwd_ex.restype = ctypes.c_int
+lib.qlora_linear_fwd_noalloc.argtypes = [_P(Nf4Struct), _vp, _i64, _vp, _vp, _i32, _f32, _vp, _vp, _vp]
+lib.qlora_linear_fwd_noalloc.restype = ctypes.c_int
 lib.qlora_linear_bwd.argtypes = [_P(Nf4Struct), _vp, _vp, _vp, _i64, _vp, _vp, _i32, _f32, _vp, _vp, _vp, _vp,
                                  _sz, _vp]
 lib.qlora_linear_bwd.restype = ctypes.c_int
@@ -220,6 +223,22 @@ def qlora_linear_fwd(q, x, a, b, alpha, y=None, u=None, ws=None, stream=None, wa
     st = lib.qlora_linear_fwd(ctypes.byref(s), _ptr(x), m, _ptr(a), _ptr(b), r, float(alpha), _ptr(y), _ptr(u),
                               _ptr(ws), ws.numel(), _stream_ptr(stream))
     _check(st, "qlora_linear_fwd")
+    return y, u
+
+
+def qlora_linear_fwd_noalloc(q, x, a, b, alpha, y=None, u=None, stream=None, want_u=True):
+    """Forward without a caller workspace (library-owned fixed scratch); returns (y, u')."""
+    torch = _torch()
+    m = x.shape[0]
+    r = a.shape[0]
+    if y is None:
+        y = torch.empty((m, q.n_out), dtype=torch.bfloat16, device=x.device)
+    if u is None and want_u:
+        u = torch.empty((m, r), dtype=torch.bfloat16, device=x.device)
+    s = q.struct()
+    st = lib.qlora_linear_fwd_noalloc(ctypes.byref(s), _ptr(x), m, _ptr(a), _ptr(b), r, float(alpha), _ptr(y),
+                                      _ptr(u), _stream_ptr(stream))
+    _check(st, "qlora_linear_fwd_noalloc")
     return y, u
 
 

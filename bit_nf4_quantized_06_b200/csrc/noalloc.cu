@@ -1,0 +1,62 @@
+// qlora_linear_fwd_noalloc: the forward for callers that cannot provide a
+// workspace.
+//
+// Some callers have no way to hand the library a scratch buffer: a runtime
+// whose device memory is entirely owned by its own pool allocator, code that
+// runs where a device allocation is forbidden or would stall other work
+// (cudaMalloc may synchronise the device), or a plain C caller without a
+// device allocator of its own. This entry point serves them with scratch
+// memory the library owns: one file-scope device array of a fixed size that
+// every GPU loading the library keeps until the process exits.
+//
+// The array's host-side name is only a stand-in for the symbol, not a device
+// address, so the host resolves the real address once per device with
+// cudaGetSymbolAddress (with that device current) and passes that pointer to
+// the existing forward as its workspace. Nothing here allocates or frees.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/qlora.h"
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of the scratch array on the current device (resolved on the
+// first call for that device). Returns nullptr on failure.
+void* scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t* q, const void* x_bf16, int64_t m,
+                                                   const void* a_bf16, const void* b_bf16, int32_t r, float alpha,
+                                                   void* y_bf16, void* u_out_bf16, void* stream) {
+  if (q == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (m == 0) {
+    return qlora_linear_fwd(q, x_bf16, m, a_bf16, b_bf16, r, alpha, y_bf16, u_out_bf16, nullptr, 0, stream);
+  }
+  const size_t need = qlora_workspace_bytes(m, q->n_out, q->k_in, r);
+  if (need == 0) return QLORA_ERR_SHAPE;
+  if (need > QLORA_NOALLOC_SCRATCH_BYTES) return QLORA_ERR_WORKSPACE;  // problem too large for the fixed scratch
+  void* ws = scratch_address();
+  if (ws == nullptr) return QLORA_ERR_CUDA;
+  return qlora_linear_fwd(q, x_bf16, m, a_bf16, b_bf16, r, alpha, y_bf16, u_out_bf16, ws,
+                          QLORA_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -133,6 +133,32 @@ QLORA_API qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t *q, const void *x
                                    float alpha, void *y_bf16, void *u_out_bf16, void *ws,
                                    size_t ws_bytes, int32_t path, void *stream);
 
+/* Size of the library-owned scratch array used by qlora_linear_fwd_noalloc
+ * (8 MiB per GPU that loads the library, held until the process exits). */
+#define QLORA_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* Forward for callers that cannot provide a workspace. The sources describe
+ * no counterpart: it is a convenience of this library. Some callers have no
+ * way to hand over scratch memory: a runtime whose device memory all belongs
+ * to its own pool, code running where a device allocation is forbidden or
+ * would stall other work (cudaMalloc may synchronise the device), or a plain
+ * C caller with no device allocator. This call computes exactly what
+ * qlora_linear_fwd computes, with the same arguments minus ws/ws_bytes, and
+ * uses instead one fixed device array of QLORA_NOALLOC_SCRATCH_BYTES owned by
+ * the library. It allocates and frees nothing.
+ *   - Problems whose qlora_workspace_bytes() exceeds the array are rejected
+ *     with QLORA_ERR_WORKSPACE before anything is launched (at r = 64 that
+ *     is from about 10,000 tokens up, depending on the weight shape).
+ *   - The first call on each device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Every call shares the one array and leaves its contents behind; no part
+ *     of it needs to start at zero (each call writes all it reads). Calls
+ *     that overlap on the GPU (other streams, other host threads) race on it:
+ *     keep them ordered, e.g. on one stream. */
+QLORA_API qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t *q, const void *x_bf16, int64_t m,
+                                                  const void *a_bf16, const void *b_bf16, int32_t r,
+                                                  float alpha, void *y_bf16, void *u_out_bf16, void *stream);
+
 /* Backward: dX [m x K] bf16 (may be NULL to skip), dA [r x K] fp32 and
  * dB [N x r] fp32 (overwritten, not accumulated). u_bf16 is the u' that the
  * forward produced ([m x r], may be NULL: then it is recomputed). No gradient
