@@ -42,6 +42,7 @@ double normal_quantile_upper(double p) {
 struct Tables {
   float cb[16];
   float mid[16];
+  double cut[16];
 };
 
 const Tables& tables() {
@@ -63,6 +64,9 @@ const Tables& tables() {
     for (int i = 0; i < 15; ++i)
       r.mid[i] = static_cast<float>((static_cast<double>(r.cb[i]) + static_cast<double>(r.cb[i + 1])) / 2.0);
     r.mid[15] = 2.0f;
+    for (int i = 0; i < 15; ++i)
+      r.cut[i] = (static_cast<double>(r.mid[i]) + static_cast<double>(std::nextafter(r.mid[i], 2.0f))) / 2.0;
+    r.cut[15] = 2.0;
     return r;
   }();
   return t;
@@ -458,7 +462,7 @@ qlora_status_t qlora_quantize_nf4(const void* w_bf16, const qlora_nf4_t* q, void
   if ((s = device_ready(nullptr)) != QLORA_OK) return s;
   const int64_t nb = q->n_out * q->k_in / kBlock;
   QuantParams qp{};
-  std::memcpy(qp.mid, tables().mid, sizeof(qp.mid));
+  std::memcpy(qp.cut, tables().cut, sizeof(qp.cut));
   const int64_t groups = cdiv(nb, kGroup);
   if (groups > 0x7FFFFFFF) return QLORA_ERR_SHAPE;
   k_quantize_nf4<<<static_cast<unsigned>(groups), 256, 0, static_cast<cudaStream_t>(stream)>>>(
@@ -551,11 +555,24 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
     gp.r64 = r64;
     gp.ldb = static_cast<int32_t>(ldb);
     std::memcpy(gp.cb, tables().cb, sizeof(gp.cb));
-    const unsigned grid = static_cast<unsigned>(cdiv(n, 16));
-    if (m <= 8)
-      k_gemv_nf4<1><<<grid, 256, 0, st>>>(gp);
-    else
-      k_gemv_nf4<2><<<grid, 256, 0, st>>>(gp);
+    // launched as a programmatic dependent of the x A^T kernel: its weight
+    // stream starts while u' is still being computed
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(cdiv(n, 16)), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = (m <= 8) ? cudaLaunchKernelEx(&cfg, k_gemv_nf4<1>, gp) : cudaLaunchKernelEx(&cfg, k_gemv_nf4<2>, gp);
+    if (e != cudaSuccess) {
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
     return launch_status();
   }
 

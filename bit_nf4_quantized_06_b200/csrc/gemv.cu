@@ -13,8 +13,11 @@
 // order, the lane's 8 consecutive weights are placed into fragment slots in
 // the order they come out of the lookup and x is fetched in the same order,
 // so no shuffle is needed. The eight warps of a CTA split K; their partial
-// fragments are summed in a fixed order in shared memory, and the LoRA term
-// is appended as r/16 further MMA steps of the same accumulator.
+// fragments are summed in a fixed order in shared memory. The LoRA term is
+// appended as r/16 further MMA steps spread over the warps; each warp fetches
+// the next chunk's codes and scale codes while it restores the current one,
+// and the kernel overlaps the small x A^T kernel before it (programmatic
+// dependent launch), waiting for u' only where it reads it.
 #include "kernels.h"
 #include "nf4_dev.cuh"
 
@@ -39,6 +42,11 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return v;
 }
 
+// Programmatic dependent launch: the consumer waits for the producer grid's
+// completion (and memory) only where it reads the producer's output.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t ld_bf16_pair(const __nv_bfloat16* row, int j, int r) {
   // (row[j], row[j+1]) with zeros past r; 2-byte loads so any r works
   const uint16_t* p = reinterpret_cast<const uint16_t*>(row);
@@ -50,7 +58,7 @@ __device__ __forceinline__ uint32_t ld_bf16_pair(const __nv_bfloat16* row, int j
 }  // namespace
 
 template <int NT>
-__global__ void __launch_bounds__(256) k_gemv_nf4(GemvParams p) {
+__global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
   constexpr int WARPS = 8;
   __shared__ float s_red[WARPS][32][NT * 4];
   const int warp = threadIdx.x >> 5;
@@ -72,29 +80,64 @@ __global__ void __launch_bounds__(256) k_gemv_nf4(GemvParams p) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[t][i] = 0.0f;
 
-  for (int64_t c = warp; c < nchunks; c += WARPS) {
-    const int64_t kb = c * 4 + qd;  // this lane's block within the row
-    const bool kv = kb < kpr;
-    uint4 a_lo = make_uint4(0, 0, 0, 0), a_hi = a_lo, b_lo = a_lo, b_hi = a_lo;
-    float sh0 = 0.0f, sh1 = 0.0f;
+  // LoRA-up fragments of this warp's rank steps (j0 = 16 * (warp + 8 i)):
+  // inputs of the call, so they are fetched before anything else
+  const __nv_bfloat16* brow0 = p.b + (v0 ? r0 : 0) * static_cast<int64_t>(p.ldb);
+  const __nv_bfloat16* brow1 = p.b + (v1 ? r1 : 0) * static_cast<int64_t>(p.ldb);
+  const int rv0 = v0 ? p.r : 0;
+  const int rv1 = v1 ? p.r : 0;
+  uint32_t la[2][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int ja = 16 * (warp + WARPS * i) + 2 * qd;
+    la[i][0] = ld_bf16_pair(brow0, ja, rv0);
+    la[i][1] = ld_bf16_pair(brow1, ja, rv1);
+    la[i][2] = ld_bf16_pair(brow0, ja + 8, rv0);
+    la[i][3] = ld_bf16_pair(brow1, ja + 8, rv1);
+  }
+
+  // one chunk = 4 blocks (256 weights) of both rows; lane (g, qd) owns block qd
+  struct Chunk {
+    uint4 a_lo, a_hi, b_lo, b_hi;
+    uint32_t q2a, q2b;
+    float sma, smb;
+  };
+  auto fetch = [&](int64_t c, Chunk& ch) {
+    const int64_t kb = c * 4 + qd;
+    const bool kv = c < nchunks && kb < kpr;
+    ch.a_lo = ch.a_hi = ch.b_lo = ch.b_hi = make_uint4(0, 0, 0, 0);
+    ch.q2a = ch.q2b = 0;
+    ch.sma = ch.smb = 0.0f;
     if (kv && v0) {
       const uint8_t* src = p.codes + r0 * row_bytes + kb * 32;
-      a_lo = ldg_stream(src);
-      a_hi = ldg_stream(src + 16);
+      ch.a_lo = ldg_stream(src);
+      ch.a_hi = ldg_stream(src + 16);
       const int64_t bi = r0 * kpr + kb;
-      sh0 = restored_scale(__ldg(p.q2 + bi), __ldg(p.smax + (bi >> 8)));
+      ch.q2a = __ldg(p.q2 + bi);
+      ch.sma = __ldg(p.smax + (bi >> 8));
     }
     if (kv && v1) {
       const uint8_t* src = p.codes + r1 * row_bytes + kb * 32;
-      b_lo = ldg_stream(src);
-      b_hi = ldg_stream(src + 16);
+      ch.b_lo = ldg_stream(src);
+      ch.b_hi = ldg_stream(src + 16);
       const int64_t bi = r1 * kpr + kb;
-      sh1 = restored_scale(__ldg(p.q2 + bi), __ldg(p.smax + (bi >> 8)));
+      ch.q2b = __ldg(p.q2 + bi);
+      ch.smb = __ldg(p.smax + (bi >> 8));
     }
-    const Nf4Table t0 = make_table(p.cb, sh0);
-    const Nf4Table t1 = make_table(p.cb, sh1);
-    const uint32_t wa[8] = {a_lo.x, a_lo.y, a_lo.z, a_lo.w, a_hi.x, a_hi.y, a_hi.z, a_hi.w};
-    const uint32_t wb[8] = {b_lo.x, b_lo.y, b_lo.z, b_lo.w, b_hi.x, b_hi.y, b_hi.z, b_hi.w};
+  };
+
+  Chunk cur, nxt;
+  fetch(warp, cur);
+  for (int64_t c = warp; c < nchunks; c += WARPS) {
+    fetch(c + WARPS, nxt);          // next chunk's loads fly while this one is restored
+    const int64_t kb = c * 4 + qd;
+    const bool kv = kb < kpr;
+    const Nf4Table t0 = make_table(p.cb, restored_scale(cur.q2a, cur.sma));
+    const Nf4Table t1 = make_table(p.cb, restored_scale(cur.q2b, cur.smb));
+    const uint32_t wa[8] = {cur.a_lo.x, cur.a_lo.y, cur.a_lo.z, cur.a_lo.w,
+                            cur.a_hi.x, cur.a_hi.y, cur.a_hi.z, cur.a_hi.w};
+    const uint32_t wb[8] = {cur.b_lo.x, cur.b_lo.y, cur.b_lo.z, cur.b_lo.w,
+                            cur.b_hi.x, cur.b_hi.y, cur.b_hi.z, cur.b_hi.w};
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
       uint32_t ra[4], rb[4];
@@ -109,6 +152,30 @@ __global__ void __launch_bounds__(256) k_gemv_nf4(GemvParams p) {
         // slots: logical k (2qd, 2qd+1) <- weights 4h+0, 4h+1; (2qd+8, 2qd+9) <- 4h+2, 4h+3
         mma_bf16_16816(acc[t], ra[0], rb[0], ra[1], rb[1], xv.x, xv.y);
         mma_bf16_16816(acc[t], ra[2], rb[2], ra[3], rb[3], xv.z, xv.w);
+      }
+    }
+    cur = nxt;
+  }
+
+  // LoRA term: sum_j u'[tok][j] B[n][j], 16 ranks per MMA step, steps spread
+  // over the warps. u' is written by the kernel launched just before this one
+  // (programmatic dependent launch), so wait for it here and only here.
+  grid_dependency_wait();
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int j0 = 16 * (warp + WARPS * i);
+    if (j0 < p.r64) {
+      const int ja = j0 + 2 * qd;
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const int tok = t * 8 + g;
+        uint32_t b0 = 0, b1 = 0;
+        if (tok < p.m) {
+          const uint32_t* urow = reinterpret_cast<const uint32_t*>(p.u + static_cast<int64_t>(tok) * p.r64);
+          b0 = urow[ja >> 1];
+          b1 = urow[(ja + 8) >> 1];
+        }
+        mma_bf16_16816(acc[t], la[i][0], la[i][1], la[i][2], la[i][3], b0, b1);
       }
     }
   }
@@ -128,30 +195,6 @@ __global__ void __launch_bounds__(256) k_gemv_nf4(GemvParams p) {
       for (int wv = 0; wv < WARPS; ++wv) v += s_red[wv][lane][t * 4 + i];
       acc[t][i] = v;
     }
-
-  // LoRA term: sum_j u'[tok][j] B[n][j], 16 ranks per MMA step
-  const __nv_bfloat16* brow0 = p.b + (v0 ? r0 : 0) * static_cast<int64_t>(p.ldb);
-  const __nv_bfloat16* brow1 = p.b + (v1 ? r1 : 0) * static_cast<int64_t>(p.ldb);
-  const int rv0 = v0 ? p.r : 0;
-  const int rv1 = v1 ? p.r : 0;
-  for (int j0 = 0; j0 < p.r64; j0 += 16) {
-    const int ja = j0 + 2 * qd;
-    const uint32_t a0 = ld_bf16_pair(brow0, ja, rv0);
-    const uint32_t a1 = ld_bf16_pair(brow1, ja, rv1);
-    const uint32_t a2 = ld_bf16_pair(brow0, ja + 8, rv0);
-    const uint32_t a3 = ld_bf16_pair(brow1, ja + 8, rv1);
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      const int tok = t * 8 + g;
-      uint32_t b0 = 0, b1 = 0;
-      if (tok < p.m) {
-        const uint32_t* urow = reinterpret_cast<const uint32_t*>(p.u + static_cast<int64_t>(tok) * p.r64);
-        b0 = urow[ja >> 1];
-        b1 = urow[(ja + 8) >> 1];
-      }
-      mma_bf16_16816(acc[t], a0, a1, a2, a3, b0, b1);
-    }
-  }
 
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
@@ -174,6 +217,7 @@ template __global__ void k_gemv_nf4<2>(GemvParams);
 // 256 threads split K in 8-element chunks, fixed-order reduction.
 __global__ void __launch_bounds__(256) k_lora_down_small(LoraDownSmallParams p) {
   __shared__ float s_part[8][16];
+  grid_dependency_trigger();   // the GEMV that consumes u' may start streaming its weights now
   const int j = blockIdx.x;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;

@@ -13,7 +13,10 @@ namespace qlora {
 extern __device__ unsigned int g_dev_status;
 
 struct QuantParams {
-  float mid[16];  // m_0..m_14: fp32 midpoints between consecutive levels; [15] unused
+  // cut[j] (j < 15): the real number halfway between m_j (the fp32 midpoint
+  // of levels j and j+1) and the next float32 above m_j; a quotient rounds
+  // to a float32 above m_j exactly when it exceeds cut[j]. cut[15] is padding.
+  double cut[16];
 };
 
 struct DequantParams {

@@ -6,7 +6,8 @@
 // 한 장에 올렸나», § "메모리 회계"):
 //   s_b   = max |w| over 64 consecutive weights of the row-major matrix
 //   q     = #{ j : fl32(w / s_b) > m_j }   (m_j = fp32 midpoints of the levels;
-//            an exact tie goes to the lower level; s_b == 0 stores level 7)
+//            an exact tie goes to the lower level; s_b == 0 stores level 7),
+//            evaluated without a division (see k_quantize_nf4)
 //   byte  = (q[2i] << 4) | q[2i+1]
 //   s_max = max s_b over 256 consecutive blocks (the last group may be short)
 //   q2    = min(255, rint_even(fl32(256 * s_b / s_max)))   (0 if s_max == 0)
@@ -41,27 +42,27 @@ __device__ __forceinline__ uint32_t abs_bits_max(uint4 v) {
   return m;
 }
 
-__device__ __forceinline__ uint32_t encode_one(float w, float s, const float* mid) {
-  if (s == 0.0f) return 7u;
-  const float x = __fdiv_rn(w, s);
-  uint32_t q = (x > mid[7]) ? 8u : 0u;
-  q += (x > mid[q + 3]) ? 4u : 0u;
-  q += (x > mid[q + 1]) ? 2u : 0u;
-  q += (x > mid[q]) ? 1u : 0u;
-  return q;
-}
-
 }  // namespace
 
+// One CTA of 256 threads per double-quantization group (see the file comment).
+//
+// Encode without dividing: for a bf16 weight w and a block scale s > 0,
+//   fl32(w / s) > m_j   <=>   w / s > m'_j   <=>   w > m'_j * s   <=>   w > RD_bf16(m'_j * s)
+// where m'_j is the midpoint between m_j and the next float32 above it.
+// Round-to-nearest sends w / s above m_j exactly when w / s exceeds that
+// midpoint; equality would need m'_j * s (a 25-bit odd significand times an
+// 8-bit one) to have at most 8 significant bits, which it cannot; m'_j * s is
+// exact in float64; and because w lies on the bf16 grid, comparing with the
+// product rounded down to that grid gives the same answer. So each block
+// computes its 15 thresholds once (two per lane of the 8 lanes that share the
+// block) and every weight is placed by a 4-step binary search over them.
 __global__ void __launch_bounds__(256) k_quantize_nf4(const uint4* __restrict__ w,
                                                       int64_t nb, uint32_t* __restrict__ codes,
                                                       uint8_t* __restrict__ q2,
                                                       float* __restrict__ smax, QuantParams qp) {
-  __shared__ float s_mid[16];
+  __shared__ float s_thr[256][17];   // per block: 15 thresholds (+ pad), row stride 17 against bank conflicts
   __shared__ uint32_t s_wmax[8];
   const int tid = threadIdx.x;
-  if (tid < 16) s_mid[tid] = qp.mid[tid];
-
   const int64_t g = blockIdx.x;
   const int64_t b0 = g * 256;
   const int nblk = static_cast<int>(nb - b0 < 256 ? nb - b0 : 256);
@@ -88,6 +89,18 @@ __global__ void __launch_bounds__(256) k_quantize_nf4(const uint4* __restrict__ 
   gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 8));
   gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 16));
   if ((tid & 31) == 0) s_wmax[tid >> 5] = gm;
+
+  // thresholds of this lane's share: j = 2 * (tid % 8) and j + 1, for each of its 8 blocks
+  const int j0 = 2 * (tid & 7);
+  const double mp0 = qp.cut[j0];
+  const double mp1 = qp.cut[j0 + 1];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int bi = (tid >> 3) + 32 * i;
+    const double sd = static_cast<double>(__uint_as_float(am[i] << 16));
+    s_thr[bi][j0] = __bfloat162float(__float2bfloat16_rd(__double2float_rd(mp0 * sd)));
+    s_thr[bi][j0 + 1] = __bfloat162float(__float2bfloat16_rd(__double2float_rd(mp1 * sd)));
+  }
   __syncthreads();
   uint32_t gmax = s_wmax[0];
 #pragma unroll
@@ -102,8 +115,8 @@ __global__ void __launch_bounds__(256) k_quantize_nf4(const uint4* __restrict__ 
       if (bi < nblk) {
         uint32_t code = 0;
         if (s_max != 0.0f) {
-          const float s = __uint_as_float(am[i] << 16);
-          const float ratio = __fdiv_rn(256.0f * s, s_max);
+          const float sb = __uint_as_float(am[i] << 16);
+          const float ratio = __fdiv_rn(256.0f * sb, s_max);
           code = static_cast<uint32_t>(min(255, __float2int_rn(ratio)));
         }
         q2[b0 + bi] = static_cast<uint8_t>(code);
@@ -115,17 +128,24 @@ __global__ void __launch_bounds__(256) k_quantize_nf4(const uint4* __restrict__ 
   for (int i = 0; i < 8; ++i) {
     const int bi = (tid >> 3) + 32 * i;
     if (bi < nblk) {
-      const float s = __uint_as_float(am[i] << 16);
+      const float* t = s_thr[bi];
+      const bool zero = (am[i] == 0);
       const uint32_t ww[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
       uint32_t word = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         // bf16 pair j holds elements 2j (low half) and 2j+1 (high half)
-        const float e0 = __uint_as_float(ww[j] << 16);
-        const float e1 = __uint_as_float(ww[j] & 0xFFFF0000u);
-        const uint32_t q0 = encode_one(e0, s, s_mid);
-        const uint32_t q1 = encode_one(e1, s, s_mid);
-        word |= ((q0 << 4) | q1) << (8 * j);
+        const float e[2] = {__uint_as_float(ww[j] << 16), __uint_as_float(ww[j] & 0xFFFF0000u)};
+        uint32_t qq[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t q = (e[h] > t[7]) ? 8u : 0u;
+          q += (e[h] > t[q + 3]) ? 4u : 0u;
+          q += (e[h] > t[q + 1]) ? 2u : 0u;
+          q += (e[h] > t[q]) ? 1u : 0u;
+          qq[h] = zero ? 7u : q;
+        }
+        word |= ((qq[0] << 4) | qq[1]) << (8 * j);
       }
       codes[chunk0 + tid + 256 * i] = word;
     }
