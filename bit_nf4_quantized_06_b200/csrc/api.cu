@@ -278,7 +278,7 @@ qlora_status_t launch_tc(int sms, cudaStream_t st, const CUtensorMap& a, const C
 // Persistent CTA-pair launch: at most `pairs` clusters of two CTAs.
 template <int AS, int NH>
 qlora_status_t launch_pair_nh(int pairs, cudaStream_t st, const CUtensorMap& b, const CUtensorMap& bl,
-                              const CUtensorMap& c, const TcParams& p) {
+                              const CUtensorMap& c, const CUtensorMap& o, const TcParams& p) {
   const int64_t tiles = static_cast<int64_t>(p.tiles_rows) * p.tiles_cols;
   if (tiles <= 0 || pairs <= 0) return QLORA_ERR_SHAPE;
   const unsigned nclusters = static_cast<unsigned>(std::min<int64_t>(tiles, pairs));
@@ -294,7 +294,7 @@ qlora_status_t launch_pair_nh(int pairs, cudaStream_t st, const CUtensorMap& b, 
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc_pair<AS, NH>, b, bl, c, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc_pair<AS, NH>, b, bl, c, o, p);
   if (e != cudaSuccess) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     cudaGetLastError();
@@ -307,15 +307,25 @@ qlora_status_t launch_pair_nh(int pairs, cudaStream_t st, const CUtensorMap& b, 
 // 256 tokens (each restored tile then feeds 512 tokens), else one.
 inline int pair_nh(int64_t m) { return m > 256 ? 2 : 1; }
 
+// The output [m x features] bf16 (row stride p.ldo) is written through TMA
+// stores when its row stride is a multiple of 16 bytes.
 template <int AS>
 qlora_status_t launch_pair(int pairs, int64_t m, cudaStream_t st, const CUtensorMap& b, const CUtensorMap& bl,
                            const CUtensorMap& c, TcParams p) {
+  CUtensorMap o = zero_map();
+  p.tma_out = 0;
+  if (p.ldo % 8 == 0 && (reinterpret_cast<uintptr_t>(p.out) & 15u) == 0) {
+    if (!map2d(&o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.out, static_cast<uint64_t>(p.rows), static_cast<uint64_t>(m),
+               static_cast<uint64_t>(p.ldo) * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+      return QLORA_ERR_CUDA;
+    p.tma_out = 1;
+  }
   if (pair_nh(m) == 2) {
     p.tiles_cols = static_cast<int32_t>(cdiv(m, 512));
-    return launch_pair_nh<AS, 2>(pairs, st, b, bl, c, p);
+    return launch_pair_nh<AS, 2>(pairs, st, b, bl, c, o, p);
   }
   p.tiles_cols = static_cast<int32_t>(cdiv(m, 256));
-  return launch_pair_nh<AS, 1>(pairs, st, b, bl, c, p);
+  return launch_pair_nh<AS, 1>(pairs, st, b, bl, c, o, p);
 }
 
 template <int AS, int BS>

@@ -91,6 +91,7 @@ struct TcParams {
   void* out;
   int64_t ldo;          // EPI_BF16_T: row stride of out [cols x ldo]; EPI_F32_ROWS: [split][rows_pad][ldo]
   int32_t rows_pad;     // EPI_F32_ROWS: rows per split slab
+  int32_t tma_out;      // pair kernel: write the output through TMA stores
 };
 
 // Persistent kernel: gridDim.x CTAs (at most one per SM) walk the tiles
@@ -120,14 +121,19 @@ constexpr int tc_smem_bytes() {
 // counts 256-row tiles and tiles_cols (256 NH)-column tiles. Launched with
 // cluster dimension 2.
 // NH = token groups of 256 per restored A tile (1 or 2).
-constexpr int pair_stages(int nh) { return nh == 1 ? 6 : 4; }
+constexpr int pair_stages(int nh) { return nh == 1 ? 5 : 4; }
+constexpr int kPairEpiStage = 4 * 2048;  // four 32 x 32 bf16 output boxes for TMA stores
 
+// tm_out: bf16 output [tokens x features] with boxes of 32 x 32 and 64-byte
+// swizzle; used when p.tma_out != 0 (row stride a multiple of 16 bytes).
 template <int AS, int NH>
 __global__ void k_tc_pair(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b_lora,
-                          const __grid_constant__ CUtensorMap tm_codes, TcParams p);
+                          const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_out,
+                          TcParams p);
 
 constexpr int tc_pair_smem_bytes(int nh) {
-  return pair_stages(nh) * (16384 + nh * 16384 + 4096) + 1024 + 256 + 2 * kScalePrefetch * 128 * 8;
+  return pair_stages(nh) * (16384 + nh * 16384 + 4096) + 1024 + 256 + 2 * kScalePrefetch * 128 * 8 +
+         kPairEpiStage;
 }
 
 // Split reductions (fixed order over splits -> deterministic).

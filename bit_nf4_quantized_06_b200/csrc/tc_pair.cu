@@ -19,10 +19,11 @@
 // Different Places": each block of W is restored to bf16 before it meets the
 // input, and gradients reach x through the restored W; W gets none.)
 //
-// With tokens on the lanes, each epilogue thread owns one output row and
-// writes 64 contiguous bytes per 32 accumulator columns (16-byte stores).
-// NH = 2 uses the whole tensor memory for one tile (its drain does not
-// overlap the next tile); NH = 1 keeps two accumulators and overlaps it.
+// With tokens on the lanes, each epilogue warp owns 32 output rows; every
+// 32 x 32 chunk goes out as one TMA tensor store from a small swizzled box.
+// NH = 2 uses the whole tensor memory for one tile, so the next tile's MMAs
+// wait until the drain has read the accumulator (not until the stores are
+// done); NH = 1 keeps two accumulators and overlaps the drain entirely.
 //
 // Warp roles in each CTA (448 threads):
 //   warp 0      TMA: this CTA's token slices (completion counted on the even
@@ -47,7 +48,8 @@ using namespace tcd;
 template <int AS, int NH>
 __global__ void __launch_bounds__(448, 1)
     k_tc_pair(const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_t_lora,
-              const __grid_constant__ CUtensorMap tm_codes, TcParams p) {
+              const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_out,
+              TcParams p) {
   constexpr int STAGES = pair_stages(NH);
   constexpr bool W_MN = (AS == A_DQ_MN);
   constexpr uint32_t W_BYTES = 16384;        // 128 features x 64 k, bf16 (restored here)
@@ -66,8 +68,9 @@ __global__ void __launch_bounds__(448, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* const ctl = smem_raw + (base - raw) + STAGES * STAGE_BYTES;
-  const uint32_t bar0 = base + STAGES * STAGE_BYTES;
+  const uint32_t epi_stage = base + STAGES * STAGE_BYTES;  // 2 KB output box per epilogue warp (1024-aligned)
+  uint8_t* const ctl = smem_raw + (base - raw) + STAGES * STAGE_BYTES + kPairEpiStage;
+  const uint32_t bar0 = epi_stage + kPairEpiStage;
   auto bar_full = [&](int s) { return bar0 + 8u * s; };                 // even CTA: token slices of both
   auto bar_codes = [&](int s) { return bar0 + 8u * (STAGES + s); };     // local code tile
   auto bar_wfull = [&](int s) { return bar0 + 8u * (2 * STAGES + s); }; // even CTA: 8 restore warps
@@ -363,9 +366,16 @@ __global__ void __launch_bounds__(448, 1)
     cp_async_wait<0>();
   } else {
     // ---------------------------------------------------------------- epilogue
+    // Each warp owns 32 token rows (its tensor-memory lane quarter). With
+    // TMA stores (row stride a multiple of 16 bytes) every 32 x 32 chunk is
+    // converted to bf16, staged in this warp's 2 KB box in the 64-byte
+    // swizzled layout (conflict-free for the row-per-lane writes) and written
+    // by one bulk tensor store; the accumulator is released as soon as its
+    // last chunk has been read. Otherwise each lane stores its row directly.
     const int quarter = warp & 3;  // TMEM lanes [32 q, 32 q + 32) belong to warp % 4
     const uint32_t acce_even0 = mapa_shared(bar_acce(0), 0);
     const bool vec_ok = (p.ldo % 8) == 0;
+    const uint32_t box = epi_stage + (warp - 10) * 2048;
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
     int tcount = 0;
     for (int tile = pair; tile < ntile_total; tile += npairs, ++tcount) {
@@ -376,49 +386,97 @@ __global__ void __launch_bounds__(448, 1)
       tc_fence_after();
       const int f0 = (tile / p.tiles_cols) * 256;   // first feature of the pair's tile
       const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-#pragma unroll 1
-      for (int h = 0; h < NH; ++h) {
-        const int token = tile_tok(tile) + 256 * h + 128 * static_cast<int>(rank) + quarter * 32 + lane;
-        __nv_bfloat16* orow = out + static_cast<int64_t>(token) * p.ldo;
-        const uint32_t taddr = tmem_base + b * TILE_COLS + h * 256 + lane_base;
-#pragma unroll 1
-        for (int ch = 0; ch < 8; ch += 2) {
-          uint32_t r0[32], r1[32];
-          tmem_ld_32x32b_x32(taddr + ch * 32, r0);
-          tmem_ld_32x32b_x32(taddr + ch * 32 + 32, r1);
-          tc_wait_ld();
-          if (token < p.cols) {
+      const uint32_t tbase = tmem_base + b * TILE_COLS + lane_base;
+      if (p.tma_out) {
+        constexpr int NCH = TILE_COLS / 32;
+        // one 32-column chunk: convert `r`, start loading chunk ch + 1 into
+        // `nx`, stage and store `r`
+        auto chunk = [&](int ch, uint32_t (&r)[32], uint32_t (&nx)[32]) {
+          uint32_t pk[16];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              const uint32_t* r = half ? r1 : r0;
-              const int fc = f0 + (ch + half) * 32;
-              if (vec_ok && fc + 32 <= p.rows) {
-                uint4* dst = reinterpret_cast<uint4*>(orow + fc);
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+          // tensor memory column c: token group c / 256, feature c % 256
+          if (ch + 1 < NCH) tmem_ld_32x32b_x32(tbase + (ch + 1) * 32, nx);
+          if (lane == 0) bulk_wait_read_all();   // the previous store has read the box
+          __syncwarp();
+          const uint32_t row = box + lane * 64;
+          const uint32_t sw = (lane >> 1) & 3;
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                  dst[v] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
-                                      pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
-                                      pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
-                                      pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+          for (int v = 0; v < 4; ++v)
+            sts128(row + ((v ^ sw) << 4), pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int h = ch / 8;
+            const int token0 = tile_tok(tile) + 256 * h + 128 * static_cast<int>(rank) + quarter * 32;
+            tma_store_2d(&tm_out, box, f0 + (ch % 8) * 32, token0);
+            bulk_commit();
+          }
+          if (ch + 1 < NCH) tc_wait_ld();
+        };
+        uint32_t ra[32], rb[32];
+        tmem_ld_32x32b_x32(tbase, ra);
+        tc_wait_ld();
+#pragma unroll 1
+        for (int ch = 0; ch < NCH; ch += 2) {
+          chunk(ch, ra, rb);
+          chunk(ch + 1, rb, ra);
+        }
+        // every column of this accumulator has been read: release it now
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader)
+            mbar_arrive(bar_acce(b));
+          else
+            mbar_arrive_cluster(acce_even0 + 8u * b);
+        }
+      } else {
+#pragma unroll 1
+        for (int h = 0; h < NH; ++h) {
+          const int token = tile_tok(tile) + 256 * h + 128 * static_cast<int>(rank) + quarter * 32 + lane;
+          __nv_bfloat16* orow = out + static_cast<int64_t>(token) * p.ldo;
+          const uint32_t taddr = tbase + h * 256;
+#pragma unroll 1
+          for (int ch = 0; ch < 8; ch += 2) {
+            uint32_t r0[32], r1[32];
+            tmem_ld_32x32b_x32(taddr + ch * 32, r0);
+            tmem_ld_32x32b_x32(taddr + ch * 32 + 32, r1);
+            tc_wait_ld();
+            if (token < p.cols) {
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+                const uint32_t* rr = half ? r1 : r0;
+                const int fc = f0 + (ch + half) * 32;
+                if (vec_ok && fc + 32 <= p.rows) {
+                  uint4* dst = reinterpret_cast<uint4*>(orow + fc);
+#pragma unroll
+                  for (int v = 0; v < 4; ++v) {
+                    dst[v] = make_uint4(pack_bf16x2(__uint_as_float(rr[8 * v + 0]), __uint_as_float(rr[8 * v + 1])),
+                                        pack_bf16x2(__uint_as_float(rr[8 * v + 2]), __uint_as_float(rr[8 * v + 3])),
+                                        pack_bf16x2(__uint_as_float(rr[8 * v + 4]), __uint_as_float(rr[8 * v + 5])),
+                                        pack_bf16x2(__uint_as_float(rr[8 * v + 6]), __uint_as_float(rr[8 * v + 7])));
+                  }
+                } else {
+#pragma unroll
+                  for (int i = 0; i < 32; ++i)
+                    if (fc + i < p.rows) orow[fc + i] = __float2bfloat16_rn(__uint_as_float(rr[i]));
                 }
-              } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                  if (fc + i < p.rows) orow[fc + i] = __float2bfloat16_rn(__uint_as_float(r[i]));
               }
             }
           }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (leader)
-          mbar_arrive(bar_acce(b));
-        else
-          mbar_arrive_cluster(acce_even0 + 8u * b);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader)
+            mbar_arrive(bar_acce(b));
+          else
+            mbar_arrive_cluster(acce_even0 + 8u * b);
+        }
       }
     }
+    if (lane == 0) bulk_wait_all();   // stores complete before the CTA's shared memory goes away
   }
 
   tc_fence_before();
@@ -432,6 +490,7 @@ __global__ void __launch_bounds__(448, 1)
 
 #define QLORA_PAIR_INST(AS, NH)                                                                         \
   template __global__ void k_tc_pair<AS, NH>(const __grid_constant__ CUtensorMap,                       \
+                                             const __grid_constant__ CUtensorMap,                       \
                                              const __grid_constant__ CUtensorMap,                       \
                                              const __grid_constant__ CUtensorMap, TcParams);
 QLORA_PAIR_INST(A_DQ_K, 1)
