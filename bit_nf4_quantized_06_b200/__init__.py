@@ -9,7 +9,7 @@ fails: there is no fallback of any kind.
 Functions carry the C names:
 
     qlora_nf4_bytes, qlora_nf4_codebook, qlora_quantize_nf4, qlora_dequantize,
-    qlora_workspace_bytes, qlora_linear_fwd, qlora_linear_fwd_ex,
+    qlora_workspace_bytes, qlora_fwd_workspace_bytes, qlora_linear_fwd, qlora_linear_fwd_ex,
     qlora_linear_fwd_noalloc, qlora_linear_bwd, qlora_device_status, qlora_status_string, qlora_version,
     qlora_launch_count
 """
@@ -20,7 +20,7 @@ import os
 __all__ = [
     "LIB_PATH", "lib", "QloraError", "NF4Weight", "Nf4Struct",
     "qlora_nf4_bytes", "qlora_nf4_codebook", "qlora_quantize_nf4", "qlora_dequantize",
-    "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_fwd_ex", "qlora_linear_fwd_noalloc",
+    "qlora_workspace_bytes", "qlora_fwd_workspace_bytes", "qlora_linear_fwd", "qlora_linear_fwd_ex", "qlora_linear_fwd_noalloc",
     "qlora_linear_bwd",
     "qlora_device_status", "qlora_status_string", "qlora_version", "qlora_launch_count",
     "FWD_AUTO", "FWD_GEMM", "FWD_GEMV",
@@ -64,6 +64,8 @@ lib.qlora_dequantize.argtypes = [_P(Nf4Struct), _vp, _vp]
 lib.qlora_dequantize.restype = ctypes.c_int
 lib.qlora_workspace_bytes.argtypes = [_i64, _i64, _i64, _i32]
 lib.qlora_workspace_bytes.restype = _sz
+lib.qlora_fwd_workspace_bytes.argtypes = [_i64, _i64, _i64, _i32]
+lib.qlora_fwd_workspace_bytes.restype = _sz
 lib.qlora_linear_fwd.argtypes = [_P(Nf4Struct), _vp, _i64, _vp, _vp, _i32, _f32, _vp, _vp, _vp, _sz, _vp]
 lib.qlora_linear_fwd.restype = ctypes.c_int
 lib.qlora_linear_fwd_ex.argtypes = [_P(Nf4Struct), _vp, _i64, _vp, _vp, _i32, _f32, _vp, _vp, _vp, _sz, _i32,
@@ -181,6 +183,10 @@ def qlora_dequantize(q, out=None, stream=None):
 
 def qlora_workspace_bytes(m, n_out, k_in, r):
     return int(lib.qlora_workspace_bytes(int(m), int(n_out), int(k_in), int(r)))
+
+
+def qlora_fwd_workspace_bytes(m, n_out, k_in, r):
+    return int(lib.qlora_fwd_workspace_bytes(int(m), int(n_out), int(k_in), int(r)))
 
 
 def _workspace(ws, m, q, r, device):

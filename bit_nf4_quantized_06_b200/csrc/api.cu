@@ -95,18 +95,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int BN, int AS, int BS, int EP>
-cudaError_t set_tc_attr() {
-  return cudaFuncSetAttribute(k_tc_gemm<BN, AS, BS, EP, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              tc_smem_bytes<BN, AS, BS, 4>());
+template <int BN, int AS, int BS>
+cudaError_t set_small_attr() {
+  return cudaFuncSetAttribute(k_tc_small<BN, AS, BS, small_stages(BN)>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              tc_small_smem_bytes<BN>());
 }
 
 template <int BN>
 cudaError_t set_small_attrs() {
   cudaError_t e;
-  if ((e = set_tc_attr<BN, A_TMA_K, B_TMA_K, EPI_F32_ROWS>()) != cudaSuccess) return e;
-  if ((e = set_tc_attr<BN, A_TMA_K, B_TMA_MN, EPI_F32_ROWS>()) != cudaSuccess) return e;
-  return set_tc_attr<BN, A_TMA_MN, B_TMA_MN, EPI_F32_ROWS>();
+  if ((e = set_small_attr<BN, A_TMA_K, B_TMA_K>()) != cudaSuccess) return e;
+  if ((e = set_small_attr<BN, A_TMA_K, B_TMA_MN>()) != cudaSuccess) return e;
+  return set_small_attr<BN, A_TMA_MN, B_TMA_MN>();
 }
 
 template <int AS, int NH>
@@ -194,13 +194,27 @@ bool map_bf16(CUtensorMap* m, const void* ptr, int64_t outer, int64_t inner, int
                CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Split count for a reduction of `ktiles` 64-wide tiles over `tiles` output tiles.
-int pick_splits(int64_t tiles, int64_t ktiles, int sms) {
-  int64_t s = sms / std::max<int64_t>(1, tiles);
-  s = std::min<int64_t>(s, ktiles);
-  s = std::min<int64_t>(s, 16);
-  s = std::max<int64_t>(s, 1);
-  const int64_t per = cdiv(ktiles, s);
+// Split count for a reduction of `ktiles` 64-wide k-tiles over `tiles`
+// output tiles of 128 x r64 on `sms` persistent CTAs. The estimate is the
+// bytes the busiest CTA moves: its tiles times (their k-tiles of operand
+// loads + one fp32 partial tile written), plus its share of the reduction's
+// re-read of all partial slabs.
+int pick_splits(int64_t tiles, int64_t ktiles, int32_t r64, int sms) {
+  tiles = std::max<int64_t>(1, tiles);
+  const double load = 16384.0 + 128.0 * r64;  // bytes per k-tile
+  const double tile_out = 512.0 * r64;        // fp32 partial tile
+  int best = 1;
+  double best_cost = 1e300;
+  for (int s = 1; s <= 16 && s <= ktiles; ++s) {
+    const double per_cta = static_cast<double>(cdiv(tiles * s, sms));
+    const double cost = per_cta * (static_cast<double>(cdiv(ktiles, s)) * load + tile_out) +
+                        static_cast<double>(s * tiles) * tile_out / sms;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  const int64_t per = cdiv(ktiles, best);
   return static_cast<int>(cdiv(ktiles, per));
 }
 
@@ -213,7 +227,7 @@ struct SmallPlan {
 SmallPlan plan_small(int64_t rows, int64_t ktiles, int32_t r64, int sms) {
   SmallPlan p;
   const int64_t tiles = cdiv(rows, 128);
-  p.splits = pick_splits(tiles, ktiles, sms);
+  p.splits = pick_splits(tiles, ktiles, r64, sms);
   p.kt_split = static_cast<int>(cdiv(ktiles, p.splits));
   p.rows_pad = tiles * 128;
   p.part_bytes = static_cast<size_t>(p.splits) * p.rows_pad * r64 * sizeof(float);
@@ -224,17 +238,20 @@ struct WsPlan {
   size_t u_pad, v_pad, b_pad, part, total;
 };
 
-WsPlan plan_ws(int64_t m, int64_t n, int64_t k, int32_t r, int sms) {
+// Workspace layout: [u_pad][v_pad][b_pad][split partials], each 256-aligned.
+// The forward needs no v_pad and only the x A^T partials.
+WsPlan plan_ws(int64_t m, int64_t n, int64_t k, int32_t r, int sms, bool fwd_only) {
   const int32_t r64 = r64_of(r);
   WsPlan w{};
   w.u_pad = al256(static_cast<size_t>(m) * r64 * 2);
-  w.v_pad = al256(static_cast<size_t>(m) * r64 * 2);
+  w.v_pad = fwd_only ? 0 : al256(static_cast<size_t>(m) * r64 * 2);
   w.b_pad = (r % 8 != 0) ? al256(static_cast<size_t>(n) * r64 * 2) : 0;
-  size_t part = 0;
-  part = std::max(part, plan_small(m, cdiv(k, 64), r64, sms).part_bytes);   // x A^T
-  part = std::max(part, plan_small(m, cdiv(n, 64), r64, sms).part_bytes);   // dY B
-  part = std::max(part, plan_small(k, cdiv(m, 64), r64, sms).part_bytes);   // dA
-  part = std::max(part, plan_small(n, cdiv(m, 64), r64, sms).part_bytes);   // dB
+  size_t part = plan_small(m, cdiv(k, 64), r64, sms).part_bytes;  // x A^T
+  if (!fwd_only) {
+    part = std::max(part, plan_small(m, cdiv(n, 64), r64, sms).part_bytes);  // dY B
+    part = std::max(part, plan_small(k, cdiv(m, 64), r64, sms).part_bytes);  // dA
+    part = std::max(part, plan_small(n, cdiv(m, 64), r64, sms).part_bytes);  // dB
+  }
   w.part = al256(part);
   w.total = w.u_pad + w.v_pad + w.b_pad + w.part + 256;
   return w;
@@ -265,13 +282,13 @@ CUtensorMap zero_map() {
 }
 
 // Persistent launch: one CTA per SM at most, each walking the tile list.
-template <int BN, int AS, int BS, int EP>
-qlora_status_t launch_tc(int sms, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& b,
-                         const CUtensorMap& bl, const CUtensorMap& c, const TcParams& p) {
-  const int64_t tiles = static_cast<int64_t>(p.tiles_rows) * p.tiles_cols * p.splits;
+template <int BN, int AS, int BS>
+qlora_status_t launch_small_bn(int sms, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& b,
+                               const SmallParams& p) {
+  const int64_t tiles = static_cast<int64_t>(p.tiles) * p.splits;
   if (tiles <= 0) return QLORA_ERR_SHAPE;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, sms));
-  k_tc_gemm<BN, AS, BS, EP, 4><<<grid, tc_threads<AS>(), tc_smem_bytes<BN, AS, BS, 4>(), st>>>(a, b, bl, c, p);
+  k_tc_small<BN, AS, BS, small_stages(BN)><<<grid, 192, tc_small_smem_bytes<BN>(), st>>>(a, b, p);
   return launch_status();
 }
 
@@ -329,61 +346,48 @@ qlora_status_t launch_pair(int pairs, int64_t m, cudaStream_t st, const CUtensor
 }
 
 template <int AS, int BS>
-qlora_status_t launch_small(int32_t r64, int sms, cudaStream_t st, const CUtensorMap& a,
-                            const CUtensorMap& b, const TcParams& p) {
-  const CUtensorMap z = zero_map();
+qlora_status_t launch_small(int32_t r64, int sms, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& b,
+                            const SmallParams& p) {
   switch (r64) {
-    case 64: return launch_tc<64, AS, BS, EPI_F32_ROWS>(sms, st, a, b, z, z, p);
-    case 128: return launch_tc<128, AS, BS, EPI_F32_ROWS>(sms, st, a, b, z, z, p);
-    case 192: return launch_tc<192, AS, BS, EPI_F32_ROWS>(sms, st, a, b, z, z, p);
-    case 256: return launch_tc<256, AS, BS, EPI_F32_ROWS>(sms, st, a, b, z, z, p);
+    case 64: return launch_small_bn<64, AS, BS>(sms, st, a, b, p);
+    case 128: return launch_small_bn<128, AS, BS>(sms, st, a, b, p);
+    case 192: return launch_small_bn<192, AS, BS>(sms, st, a, b, p);
+    case 256: return launch_small_bn<256, AS, BS>(sms, st, a, b, p);
     default: return QLORA_ERR_SHAPE;
   }
 }
 
-qlora_status_t launch_reduce(const ReduceParams& rp, int sms, cudaStream_t st) {
-  const int64_t total = static_cast<int64_t>(rp.rows) * (rp.mode == 0 ? rp.ld : rp.cols);
-  const int blocks = static_cast<int>(std::min<int64_t>(cdiv(total, 256), int64_t(sms) * 8));
-  k_reduce_splits<<<std::max(blocks, 1), 256, 0, st>>>(rp);
-  return launch_status();
-}
-
-// out_pad[rows x r64] = bf16(scale * (A_rows . B)) for a TMA-fed LoRA product
-// with the reduction over `kdim` (split over the grid's z).
+// A TMA-fed LoRA product over a reduction of length `kdim`: split-K partial
+// slabs in `part`, then the fixed-order reduction writes mode 0 bf16(scale *
+// .) to out_pad [rows x r64] (and out_c [rows x r] when set), mode 1 fp32
+// out_f [rows x r], mode 2 fp32 out_f [r x rows] (transposed).
 template <int AS, int BS>
 qlora_status_t lora_product(const CUtensorMap& ma, const CUtensorMap& mb, int64_t rows, int64_t kdim,
-                            int32_t r, float scale, int reduce_mode, __nv_bfloat16* out_pad,
-                            __nv_bfloat16* out_c, float* out_f, float* part, int sms,
-                            cudaStream_t st) {
+                            int32_t r, float scale, int mode, __nv_bfloat16* out_pad, __nv_bfloat16* out_c,
+                            float* out_f, float* part, int sms, cudaStream_t st) {
   const int32_t r64 = r64_of(r);
   const SmallPlan sp = plan_small(rows, cdiv(kdim, 64), r64, sms);
-  TcParams p{};
+  SmallParams p{};
   p.rows = static_cast<int32_t>(rows);
-  p.cols = r64;
-  p.kt_main = static_cast<int32_t>(cdiv(kdim, 64));
-  p.kt_lora = 0;
-  p.kt_split = sp.kt_split;
-  p.tiles_rows = static_cast<int32_t>(cdiv(rows, 128));
-  p.tiles_cols = 1;
-  p.splits = sp.splits;
-  p.out = part;
-  p.ldo = r64;
   p.rows_pad = static_cast<int32_t>(sp.rows_pad);
+  p.ld = r64;
+  p.cols = r;
+  p.tiles = static_cast<int32_t>(cdiv(rows, 128));
+  p.kt_main = static_cast<int32_t>(cdiv(kdim, 64));
+  p.kt_split = sp.kt_split;
+  p.splits = sp.splits;
+  p.part = part;
+  p.scale = scale;
+  p.mode = mode;
+  p.out_pad = out_pad;
+  p.out_c = out_c;
+  p.out_f = out_f;
   qlora_status_t s = launch_small<AS, BS>(r64, sms, st, ma, mb, p);
   if (s != QLORA_OK) return s;
-  ReduceParams rp{};
-  rp.part = part;
-  rp.splits = sp.splits;
-  rp.rows = static_cast<int32_t>(rows);
-  rp.rows_pad = static_cast<int32_t>(sp.rows_pad);
-  rp.ld = r64;
-  rp.cols = r;
-  rp.scale = scale;
-  rp.out_pad = out_pad;
-  rp.out_c = out_c;
-  rp.out_f = out_f;
-  rp.mode = reduce_mode;
-  return launch_reduce(rp, sms, st);
+  const int total = p.rows * (r64 / 4);
+  const int blocks = static_cast<int>(std::min<int64_t>(cdiv(total, 256), int64_t(sms) * 8));
+  k_reduce_splits<<<std::max(blocks, 1), 256, 0, st>>>(p);
+  return launch_status();
 }
 
 struct LinearArgs {
@@ -395,7 +399,7 @@ struct LinearArgs {
   size_t ws_bytes;
 };
 
-qlora_status_t check_linear(const LinearArgs& a, int sms) {
+qlora_status_t check_linear(const LinearArgs& a, int sms, bool fwd_only) {
   qlora_status_t s = check_nf4(a.q);
   if (s != QLORA_OK) return s;
   if (a.m < 0 || a.m > (int64_t(1) << 31) - 1) return QLORA_ERR_SHAPE;
@@ -403,7 +407,7 @@ qlora_status_t check_linear(const LinearArgs& a, int sms) {
   if (!std::isfinite(a.alpha)) return QLORA_ERR_INVALID_ARG;
   if (a.m == 0) return QLORA_OK;
   if (a.ws == nullptr || !aligned16(a.ws)) return a.ws == nullptr ? QLORA_ERR_WORKSPACE : QLORA_ERR_ALIGNMENT;
-  if (a.ws_bytes < plan_ws(a.m, a.q->n_out, a.q->k_in, a.r, sms).total) return QLORA_ERR_WORKSPACE;
+  if (a.ws_bytes < plan_ws(a.m, a.q->n_out, a.q->k_in, a.r, sms, fwd_only).total) return QLORA_ERR_WORKSPACE;
   return QLORA_OK;
 }
 
@@ -452,8 +456,8 @@ size_t qlora_nf4_bytes(int64_t n_out, int64_t k_in, int32_t dq_group, size_t out
   return b0 + b1 + b2;
 }
 
-size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r) {
-  if (m < 0 || n_out <= 0 || k_in <= 0 || r < 1 || r > kMaxRank) return 0;
+namespace {
+int current_sms() {
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) {
@@ -461,7 +465,18 @@ size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r) 
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
   }
   cudaGetLastError();
-  return plan_ws(std::max<int64_t>(m, 1), n_out, k_in, r, sms).total;
+  return sms;
+}
+}  // namespace
+
+size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r) {
+  if (m < 0 || n_out <= 0 || k_in <= 0 || r < 1 || r > kMaxRank) return 0;
+  return plan_ws(std::max<int64_t>(m, 1), n_out, k_in, r, current_sms(), false).total;
+}
+
+size_t qlora_fwd_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r) {
+  if (m < 0 || n_out <= 0 || k_in <= 0 || r < 1 || r > kMaxRank) return 0;
+  return plan_ws(std::max<int64_t>(m, 1), n_out, k_in, r, current_sms(), true).total;
 }
 
 qlora_status_t qlora_quantize_nf4(const void* w_bf16, const qlora_nf4_t* q, void* stream) {
@@ -507,7 +522,7 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
   if (path < QLORA_FWD_AUTO || path > QLORA_FWD_GEMV) return QLORA_ERR_INVALID_ARG;
   if ((s = device_ready(&sms, &pairs)) != QLORA_OK) return s;
   const LinearArgs la{q, m, r, alpha, ws, ws_bytes};
-  if ((s = check_linear(la, sms)) != QLORA_OK) return s;
+  if ((s = check_linear(la, sms, true)) != QLORA_OK) return s;
   if (m == 0) return QLORA_OK;
   if (x == nullptr || a == nullptr || b == nullptr || y == nullptr) return QLORA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(a) || !aligned16(b) || !aligned16(y) || (u_out && !aligned16(u_out)))
@@ -519,7 +534,7 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
   const int64_t n = q->n_out, k = q->k_in;
   const int32_t r64 = r64_of(r);
   const float sc = alpha / static_cast<float>(r);
-  const WsPlan wp = plan_ws(m, n, k, r, sms);
+  const WsPlan wp = plan_ws(m, n, k, r, sms, true);
   uint8_t* wsb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
   __nv_bfloat16* u_pad = reinterpret_cast<__nv_bfloat16*>(wsb);
   __nv_bfloat16* b_pad = reinterpret_cast<__nv_bfloat16*>(wsb + wp.u_pad + wp.v_pad);
@@ -637,7 +652,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
   if (s != QLORA_OK) return s;
   if ((s = device_ready(&sms, &pairs)) != QLORA_OK) return s;
   const LinearArgs la{q, m, r, alpha, ws, ws_bytes};
-  if ((s = check_linear(la, sms)) != QLORA_OK) return s;
+  if ((s = check_linear(la, sms, false)) != QLORA_OK) return s;
   if (x == nullptr || dy == nullptr || a == nullptr || b == nullptr || da == nullptr || db == nullptr)
     return QLORA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(dy) || !aligned16(a) || !aligned16(b) || !aligned16(da) || !aligned16(db) ||
@@ -655,7 +670,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
   }
   const int32_t r64 = r64_of(r);
   const float sc = alpha / static_cast<float>(r);
-  const WsPlan wp = plan_ws(m, n, k, r, sms);
+  const WsPlan wp = plan_ws(m, n, k, r, sms, false);
   uint8_t* wsb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
   __nv_bfloat16* u_pad = reinterpret_cast<__nv_bfloat16*>(wsb);
   __nv_bfloat16* v_pad = reinterpret_cast<__nv_bfloat16*>(wsb + wp.u_pad);

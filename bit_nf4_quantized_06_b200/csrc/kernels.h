@@ -61,10 +61,10 @@ __global__ void k_gemv_nf4(GemvParams p);
 __global__ void k_lora_down_small(LoraDownSmallParams p);
 
 // ------------------------------------------------------------ tensor-core GEMM engine
-// Operand sources of the generic tcgen05 kernel.
+// Operand sources: A from TMA (K- or MN-major), or the restored NF4 weight
+// (K-major for the forward, MN-major for dX); B from TMA.
 enum ASrc : int { A_TMA_K = 0, A_TMA_MN = 1, A_DQ_K = 2, A_DQ_MN = 3 };
 enum BSrc : int { B_TMA_K = 0, B_TMA_MN = 1 };
-enum Epi : int { EPI_BF16_T = 0, EPI_F32_ROWS = 1 };
 
 struct TcParams {
   int32_t rows;         // extent of the D rows (TMEM lanes) over the whole grid
@@ -89,32 +89,47 @@ struct TcParams {
   int32_t lora_r;       // valid extent of the LoRA rank
   // output
   void* out;
-  int64_t ldo;          // EPI_BF16_T: row stride of out [cols x ldo]; EPI_F32_ROWS: [split][rows_pad][ldo]
-  int32_t rows_pad;     // EPI_F32_ROWS: rows per split slab
+  int64_t ldo;          // pair kernel: row stride of out [cols x ldo]; small kernel: slabs [split][rows_pad][ldo]
+  int32_t rows_pad;     // small kernel: rows per split slab
   int32_t tma_out;      // pair kernel: write the output through TMA stores
 };
 
-// Persistent kernel: gridDim.x CTAs (at most one per SM) walk the tiles
-// blockIdx.x, blockIdx.x + gridDim.x, ...
-template <int BN, int AS, int BS, int EP, int STAGES>
-__global__ void k_tc_gemm(const __grid_constant__ CUtensorMap tm_a,
-                          const __grid_constant__ CUtensorMap tm_b,
-                          const __grid_constant__ CUtensorMap tm_b_lora,
-                          const __grid_constant__ CUtensorMap tm_codes, TcParams p);
-
-constexpr int kScalePrefetch = 4;  // k-tiles of scale codes fetched ahead by each A-producer thread
-
-template <int AS>
-constexpr bool tc_dq() { return AS == A_DQ_K || AS == A_DQ_MN; }
-
-template <int AS>
-constexpr int tc_threads() { return tc_dq<AS>() ? 448 : 192; }
+// TMA-fed tcgen05 GEMM for the small LoRA products: persistent CTAs (at most
+// one per SM) walk tile = row tile * splits + split and write fp32 partial
+// slabs part[split][rows_pad][ld]; k_reduce_splits finishes them.
+struct SmallParams {
+  int32_t rows;          // output rows
+  int32_t rows_pad;      // tiles * 128
+  int32_t ld;            // padded width r64 = BN (slab row stride; mode 0 out_pad row stride)
+  int32_t cols;          // valid output columns r
+  int32_t tiles;         // 128-row tiles
+  int32_t kt_main;       // 64-wide k-tiles of the reduction
+  int32_t kt_split;      // k-tiles per split
+  int32_t splits;
+  float* part;           // [splits][rows_pad][ld] fp32
+  float scale;
+  int32_t mode;          // 0: bf16 out_pad [rows x ld] and out_c [rows x cols] (if set)
+                         // 1: fp32 out_f [rows x cols]; 2: fp32 out_f [cols x rows]
+  __nv_bfloat16* out_pad;
+  __nv_bfloat16* out_c;
+  float* out_f;
+};
 
 template <int BN, int AS, int BS, int STAGES>
-constexpr int tc_smem_bytes() {
-  return STAGES * (16384 + BN * 128 + (tc_dq<AS>() ? 4096 : 0)) + 1024 + 256 +
-         (tc_dq<AS>() ? 2 * kScalePrefetch * 128 * 8 : 0);
+__global__ void k_tc_small(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                           SmallParams p);
+
+// as many pipeline stages as fit beside the control block, at most eight
+constexpr int small_stages(int bn) {
+  return (200 * 1024) / (16384 + bn * 128) > 8 ? 8 : (200 * 1024) / (16384 + bn * 128);
 }
+
+template <int BN>
+constexpr int tc_small_smem_bytes() {
+  return small_stages(BN) * (16384 + BN * 128) + 1024 + 256;
+}
+
+constexpr int kScalePrefetch = 4;  // k-tiles of scale codes fetched ahead by each restore thread
 
 // CTA-pair (cta_group::2) fused restore + GEMM for the forward (A_DQ_K) and
 // dX (A_DQ_MN): clusters of two CTAs walk 256 x (256 NH) tiles; tiles_rows
@@ -136,17 +151,7 @@ constexpr int tc_pair_smem_bytes(int nh) {
          kPairEpiStage;
 }
 
-// Split reductions (fixed order over splits -> deterministic).
-struct ReduceParams {
-  const float* part;        // [splits][rows_pad][ld]
-  int32_t splits, rows, rows_pad, ld, cols;
-  float scale;
-  __nv_bfloat16* out_pad;   // mode 0: bf16 [rows x ld]   (all ld columns)
-  __nv_bfloat16* out_c;     // mode 0: bf16 [rows x cols] (may be null)
-  float* out_f;             // mode 1: fp32 [rows x cols]; mode 2: fp32 [cols x rows] (transposed)
-  int32_t mode;
-};
-__global__ void k_reduce_splits(ReduceParams p);
+__global__ void k_reduce_splits(SmallParams p);
 
 // Zero-padded copy of a [rows x r] bf16 matrix into [rows x r64].
 __global__ void k_pad_cols(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,

@@ -52,7 +52,7 @@ extern "C" qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t* q, const v
   if (m == 0) {
     return qlora_linear_fwd(q, x_bf16, m, a_bf16, b_bf16, r, alpha, y_bf16, u_out_bf16, nullptr, 0, stream);
   }
-  const size_t need = qlora_workspace_bytes(m, q->n_out, q->k_in, r);
+  const size_t need = qlora_fwd_workspace_bytes(m, q->n_out, q->k_in, r);
   if (need == 0) return QLORA_ERR_SHAPE;
   if (need > QLORA_NOALLOC_SCRATCH_BYTES) return QLORA_ERR_WORKSPACE;  // problem too large for the fixed scratch
   void* ws = scratch_address();

@@ -115,8 +115,14 @@ QLORA_API qlora_status_t qlora_quantize_nf4(const void *w_bf16, const qlora_nf4_
 QLORA_API qlora_status_t qlora_dequantize(const qlora_nf4_t *q, void *w_bf16_out, void *stream);
 
 /* Workspace bytes that qlora_linear_fwd / _bwd need for these sizes (an
- * upper bound that covers both calls and every forward path). */
+ * upper bound that covers both calls and every forward path). 0 for
+ * arguments out of range. The size depends on the SM count of the current
+ * device: ask with the device current that the calls will run on. */
 QLORA_API size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r);
+
+/* Workspace bytes that qlora_linear_fwd alone needs (at most
+ * qlora_workspace_bytes for the same sizes). */
+QLORA_API size_t qlora_fwd_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r);
 
 /* Forward: y [m x N] = x W_hat^T + s (x A^T) B^T, bf16 out, fp32 accumulate.
  * x [m x K], A [r x K], B [N x r] bf16 (device); 1 <= r <= 256; m >= 0
@@ -146,9 +152,12 @@ QLORA_API qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t *q, const void *x
  * qlora_linear_fwd computes, with the same arguments minus ws/ws_bytes, and
  * uses instead one fixed device array of QLORA_NOALLOC_SCRATCH_BYTES owned by
  * the library. It allocates and frees nothing.
- *   - Problems whose qlora_workspace_bytes() exceeds the array are rejected
- *     with QLORA_ERR_WORKSPACE before anything is launched (at r = 64 that
- *     is from about 10,000 tokens up, depending on the weight shape).
+ *   - Problems whose qlora_fwd_workspace_bytes() exceeds the array are
+ *     rejected with QLORA_ERR_WORKSPACE before anything is launched. Ask
+ *     that function beforehand: the need follows the split plan and is not
+ *     monotone in m. On a 148-SM B200 at r <= 64 every m up to 2,304 tokens
+ *     fits for 4096 x 11008 and 8192 x 22016 weights of either orientation
+ *     (up to 6,272 for 11008 x 4096 and 4096 x 4096); at r = 256 up to 384.
  *   - The first call on each device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
  *   - Every call shares the one array and leaves its contents behind; no part

@@ -67,6 +67,15 @@ def test_workspace_bytes_positive_and_monotone(q):
     assert q.qlora_workspace_bytes(16, 512, 512, 257) == 0
 
 
+def test_forward_workspace_within_full_workspace(q):
+    for m, n, k, r in [(1, 4096, 4096, 64), (300, 512, 512, 8), (4096, 11008, 4096, 64),
+                       (2048, 8192, 22016, 256), (50000, 22016, 8192, 16)]:
+        f = q.qlora_fwd_workspace_bytes(m, n, k, r)
+        assert 0 < f <= q.qlora_workspace_bytes(m, n, k, r)
+    assert q.qlora_fwd_workspace_bytes(16, 512, 512, 0) == 0
+    assert q.qlora_fwd_workspace_bytes(-1, 512, 512, 8) == 0
+
+
 def test_argument_validation_before_any_launch(q):
     lib = q.lib
     s = q.Nf4Struct(512, 512, 64, 256, 0, 0, 0)           # null buffers

@@ -54,7 +54,7 @@ def test_noalloc_forward_matches_workspace_forward_twice(q, n, k, m, r):
 def test_noalloc_rejects_problems_beyond_its_scratch(q):
     n, k, r = 256, 4096, 64
     m = 200000
-    assert q.qlora_workspace_bytes(m, n, k, r) > 8 * 1024 * 1024
+    assert q.qlora_fwd_workspace_bytes(m, n, k, r) > 8 * 1024 * 1024
     s = q.Nf4Struct(n, k, 64, 256, 256, 256, 256)      # never dereferenced: rejected first
     st = q.lib.qlora_linear_fwd_noalloc(ctypes.byref(s), ctypes.c_void_p(256), m, ctypes.c_void_p(256),
                                         ctypes.c_void_p(256), r, 16.0, ctypes.c_void_p(256), None, None)
