@@ -11,7 +11,7 @@ Functions carry the C names:
     qlora_nf4_bytes, qlora_nf4_codebook, qlora_quantize_nf4, qlora_dequantize,
     qlora_workspace_bytes, qlora_fwd_workspace_bytes, qlora_linear_fwd, qlora_linear_fwd_ex,
     qlora_linear_fwd_noalloc, qlora_linear_bwd, qlora_device_status, qlora_status_string, qlora_version,
-    qlora_launch_count
+    qlora_launch_count, qlora_selftest_wait_timeout
 """
 
 import ctypes
@@ -23,6 +23,7 @@ __all__ = [
     "qlora_workspace_bytes", "qlora_fwd_workspace_bytes", "qlora_linear_fwd", "qlora_linear_fwd_ex", "qlora_linear_fwd_noalloc",
     "qlora_linear_bwd",
     "qlora_device_status", "qlora_status_string", "qlora_version", "qlora_launch_count",
+    "qlora_selftest_wait_timeout",
     "FWD_AUTO", "FWD_GEMM", "FWD_GEMV",
 ]
 
@@ -82,6 +83,8 @@ lib.qlora_status_string.argtypes = [ctypes.c_int]
 lib.qlora_status_string.restype = ctypes.c_char_p
 lib.qlora_version.argtypes = []
 lib.qlora_version.restype = _i32
+lib.qlora_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _vp]
+lib.qlora_selftest_wait_timeout.restype = ctypes.c_int
 lib.qlora_launch_count.argtypes = []
 lib.qlora_launch_count.restype = ctypes.c_uint64
 
@@ -272,3 +275,9 @@ def qlora_device_status(stream=None):
     bits = ctypes.c_uint32(0)
     st = lib.qlora_device_status(_stream_ptr(stream), ctypes.byref(bits))
     return int(st), int(bits.value)
+
+
+def qlora_selftest_wait_timeout(limit_us, stream=None):
+    """Launch the bounded-wait self test (a wait that nothing completes); the
+    timeout shows up in the next qlora_device_status()."""
+    _check(lib.qlora_selftest_wait_timeout(int(limit_us), _stream_ptr(stream)), "qlora_selftest_wait_timeout")

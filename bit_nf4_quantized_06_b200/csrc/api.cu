@@ -12,6 +12,7 @@
 
 #include "../../include/qlora.h"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace qlora {
 namespace {
@@ -563,7 +564,20 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
     lp.r = r;
     lp.r64 = r64;
     lp.s = sc;
-    k_lora_down_small<<<r64, 256, 0, st>>>(lp);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t dcfg = {};
+    dcfg.gridDim = dim3(static_cast<unsigned>(r64), 1, 1);
+    dcfg.blockDim = dim3(256, 1, 1);
+    dcfg.stream = st;
+    dcfg.attrs = attr;
+    dcfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&dcfg, k_lora_down_small, lp) != cudaSuccess) {
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
     if ((s = launch_status()) != QLORA_OK) return s;
     GemvParams gp{};
     gp.codes = q->codes;
@@ -583,9 +597,6 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
     // launched as a programmatic dependent of the x A^T kernel: its weight
     // stream starts while u' is still being computed
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(static_cast<unsigned>(cdiv(n, 16)), 1, 1);
     cfg.blockDim = dim3(256, 1, 1);
     cfg.dynamicSmemBytes = 0;
@@ -768,6 +779,20 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
     if (s != QLORA_OK) return s;
   }
   return QLORA_OK;
+}
+
+static_assert(QLORA_DEV_TIMEOUT_PRODUCER == QLORA_STATUS_BIT_PRODUCER && QLORA_DEV_TIMEOUT_MMA == QLORA_STATUS_BIT_MMA &&
+                  QLORA_DEV_TIMEOUT_APROD == QLORA_STATUS_BIT_RESTORE && QLORA_DEV_TIMEOUT_EPI == QLORA_STATUS_BIT_EPILOGUE &&
+                  QLORA_DEV_TIMEOUT_SELFTEST == QLORA_STATUS_BIT_SELFTEST,
+              "device status bits match the header");
+
+qlora_status_t qlora_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+  int sms = 0, pairs = 0;
+  qlora_status_t s = device_ready(&sms, &pairs);
+  if (s != QLORA_OK) return s;
+  const uint64_t us = std::min<uint64_t>(std::max<uint32_t>(limit_us, 1u), 2000000u);
+  k_selftest_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(us * 1000ull);
+  return launch_status();
 }
 
 qlora_status_t qlora_device_status(void* stream, uint32_t* bits) {

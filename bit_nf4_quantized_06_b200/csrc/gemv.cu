@@ -16,8 +16,11 @@
 // fragments are summed in a fixed order in shared memory. The LoRA term is
 // appended as r/16 further MMA steps spread over the warps; each warp fetches
 // the next chunk's codes and scale codes while it restores the current one,
-// and the kernel overlaps the small x A^T kernel before it (programmatic
-// dependent launch), waiting for u' only where it reads it.
+// and both kernels use programmatic dependent launch: x A^T starts while the
+// kernel before it drains and waits for it before reading anything; the GEMV
+// starts as soon as x A^T has started, requests its first weight chunks and
+// then waits for x A^T (and so for everything before it) to complete before
+// it reads x or u'.
 #include "kernels.h"
 #include "nf4_dev.cuh"
 
@@ -126,10 +129,15 @@ __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
     }
   };
 
+  // The packed weight and B are not written by the kernel launched just
+  // before this one (x A^T), so their first two chunks are requested before
+  // waiting for it; x and u' are read only after the wait.
   Chunk cur, nxt;
   fetch(warp, cur);
+  fetch(warp + WARPS, nxt);
+  grid_dependency_trigger();
+  grid_dependency_wait();
   for (int64_t c = warp; c < nchunks; c += WARPS) {
-    fetch(c + WARPS, nxt);          // next chunk's loads fly while this one is restored
     const int64_t kb = c * 4 + qd;
     const bool kv = kb < kpr;
     const Nf4Table t0 = make_table(p.cb, restored_scale(cur.q2a, cur.sma));
@@ -155,12 +163,11 @@ __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
       }
     }
     cur = nxt;
+    fetch(c + 2 * WARPS, nxt);      // loads of the chunk after next fly while the next one is restored
   }
 
   // LoRA term: sum_j u'[tok][j] B[n][j], 16 ranks per MMA step, steps spread
-  // over the warps. u' is written by the kernel launched just before this one
-  // (programmatic dependent launch), so wait for it here and only here.
-  grid_dependency_wait();
+  // over the warps.
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int j0 = 16 * (warp + WARPS * i);
@@ -218,6 +225,7 @@ template __global__ void k_gemv_nf4<2>(GemvParams);
 __global__ void __launch_bounds__(256) k_lora_down_small(LoraDownSmallParams p) {
   __shared__ float s_part[8][16];
   grid_dependency_trigger();   // the GEMV that consumes u' may start streaming its weights now
+  grid_dependency_wait();      // x (and A) may come from the kernel before this one
   const int j = blockIdx.x;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;

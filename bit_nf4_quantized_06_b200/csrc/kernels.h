@@ -153,6 +153,8 @@ constexpr int tc_pair_smem_bytes(int nh) {
 
 __global__ void k_reduce_splits(SmallParams p);
 
+__global__ void k_selftest_wait(uint64_t limit_ns);
+
 // Zero-padded copy of a [rows x r] bf16 matrix into [rows x r64].
 __global__ void k_pad_cols(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
                            int64_t rows, int32_t r, int32_t r64);

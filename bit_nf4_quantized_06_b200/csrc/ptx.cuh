@@ -20,6 +20,7 @@
 #define QLORA_DEV_TIMEOUT_MMA      0x2u
 #define QLORA_DEV_TIMEOUT_APROD    0x4u
 #define QLORA_DEV_TIMEOUT_EPI      0x8u
+#define QLORA_DEV_TIMEOUT_SELFTEST 0x10u
 
 namespace qlora {
 

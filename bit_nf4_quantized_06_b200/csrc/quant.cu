@@ -180,4 +180,24 @@ __global__ void __launch_bounds__(256) k_dequantize_nf4(const uint32_t* __restri
   }
 }
 
+// Failure-detection self test: one thread waits on a shared-memory barrier
+// that expects one arrival nobody makes. The wait is bounded by `limit_ns`
+// of global time; when it runs out the kernel records the self-test bit and
+// returns, with nothing in flight (no copies, no tensor memory).
+__global__ void __launch_bounds__(32) k_selftest_wait(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    fence_mbar_init();
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(b, 0)) {
+      if (globaltimer_ns() - t0 > limit_ns) {
+        atomicOr(&g_dev_status, QLORA_DEV_TIMEOUT_SELFTEST);
+        break;
+      }
+    }
+  }
+}
+
 }  // namespace qlora

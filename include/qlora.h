@@ -182,6 +182,23 @@ QLORA_API qlora_status_t qlora_linear_bwd(const qlora_nf4_t *q, const void *x_bf
  * bounded wait; *bits, if non-NULL, gets which role), or QLORA_ERR_CUDA. */
 QLORA_API qlora_status_t qlora_device_status(void *stream, uint32_t *bits);
 
+/* Status bits that qlora_device_status() may return in *bits: which kind
+ * of wait ran out of time. */
+#define QLORA_STATUS_BIT_PRODUCER 0x1u  /* a load producer waited for a free stage */
+#define QLORA_STATUS_BIT_MMA      0x2u  /* the MMA issuer waited for operands      */
+#define QLORA_STATUS_BIT_RESTORE  0x4u  /* a restore warp waited for codes/scales  */
+#define QLORA_STATUS_BIT_EPILOGUE 0x8u  /* the epilogue waited for an accumulator  */
+#define QLORA_STATUS_BIT_SELFTEST 0x10u /* qlora_selftest_wait_timeout             */
+
+/* Diagnostic for the failure-detection path (not part of the method): one
+ * tiny kernel waits on a shared-memory barrier that nothing ever completes,
+ * gives up after limit_us microseconds (clamped to [1, 2000000]), sets
+ * QLORA_STATUS_BIT_SELFTEST and returns normally. The CUDA context stays
+ * usable; qlora_device_status() then returns QLORA_ERR_TIMEOUT with that bit.
+ * Lets a caller check that its error handling sees a timed-out wait without
+ * any GPU fault. */
+QLORA_API qlora_status_t qlora_selftest_wait_timeout(uint32_t limit_us, void *stream);
+
 /* Static description of a status code. */
 QLORA_API const char *qlora_status_string(qlora_status_t s);
 
