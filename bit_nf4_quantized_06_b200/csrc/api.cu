@@ -568,12 +568,16 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t dcfg = {};
-    dcfg.gridDim = dim3(static_cast<unsigned>(r64), 1, 1);
-    dcfg.blockDim = dim3(256, 1, 1);
+    // m = 1: 16 CTAs of 16 warps, four ranks per CTA per pass; else one CTA of 4 warps per rank
+    dcfg.gridDim = dim3(static_cast<unsigned>(m == 1 ? std::min<int64_t>(16, cdiv(r64, 4)) : r64), 1, 1);
+    dcfg.blockDim = dim3(m == 1 ? 512 : 128, 1, 1);
     dcfg.stream = st;
     dcfg.attrs = attr;
     dcfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&dcfg, k_lora_down_small, lp) != cudaSuccess) {
+    const cudaError_t de = (m == 1)   ? cudaLaunchKernelEx(&dcfg, k_lora_down_small<1>, lp)
+                           : (m <= 8) ? cudaLaunchKernelEx(&dcfg, k_lora_down_small<8>, lp)
+                                      : cudaLaunchKernelEx(&dcfg, k_lora_down_small<16>, lp);
+    if (de != cudaSuccess) {
       g_launches.fetch_add(1, std::memory_order_relaxed);
       cudaGetLastError();
       return QLORA_ERR_CUDA;

@@ -16,11 +16,10 @@
 // fragments are summed in a fixed order in shared memory. The LoRA term is
 // appended as r/16 further MMA steps spread over the warps; each warp fetches
 // the next chunk's codes and scale codes while it restores the current one,
-// and both kernels use programmatic dependent launch: x A^T starts while the
-// kernel before it drains and waits for it before reading anything; the GEMV
-// starts as soon as x A^T has started, requests its first weight chunks and
-// then waits for x A^T (and so for everything before it) to complete before
-// it reads x or u'.
+// and both kernels use programmatic dependent launch: x A^T may launch while
+// the kernel before it drains, waits for it, and then lets the GEMV start;
+// the GEMV streams the whole weight while x A^T runs beside it and waits for
+// x A^T only before the LoRA-up step that reads u'.
 #include "kernels.h"
 #include "nf4_dev.cuh"
 
@@ -129,14 +128,13 @@ __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
     }
   };
 
-  // The packed weight and B are not written by the kernel launched just
-  // before this one (x A^T), so their first two chunks are requested before
-  // waiting for it; x and u' are read only after the wait.
+  // x A^T, the kernel launched just before this one, starts only after all
+  // earlier work is complete and writes nothing but u'; so everything except
+  // u' may be read at once, and u' only after waiting for that kernel.
   Chunk cur, nxt;
   fetch(warp, cur);
   fetch(warp + WARPS, nxt);
   grid_dependency_trigger();
-  grid_dependency_wait();
   for (int64_t c = warp; c < nchunks; c += WARPS) {
     const int64_t kb = c * 4 + qd;
     const bool kv = kb < kpr;
@@ -167,7 +165,8 @@ __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
   }
 
   // LoRA term: sum_j u'[tok][j] B[n][j], 16 ranks per MMA step, steps spread
-  // over the warps.
+  // over the warps. u' comes from the kernel in front: wait for it here.
+  grid_dependency_wait();
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int j0 = 16 * (warp + WARPS * i);
@@ -220,61 +219,83 @@ __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
 template __global__ void k_gemv_nf4<1>(GemvParams);
 template __global__ void k_gemv_nf4<2>(GemvParams);
 
-// u'[m][j] = bf16(s * sum_k x[m][k] A[j][k]) for M <= 16: one CTA per rank j,
-// 256 threads split K in 8-element chunks, fixed-order reduction.
-__global__ void __launch_bounds__(256) k_lora_down_small(LoraDownSmallParams p) {
-  __shared__ float s_part[8][16];
-  grid_dependency_trigger();   // the GEMV that consumes u' may start streaming its weights now
-  grid_dependency_wait();      // x (and A) may come from the kernel before this one
-  const int j = blockIdx.x;
+// u'[m][j] = bf16(s * sum_k x[m][k] A[j][k]) for M <= 16 (the decode LoRA
+// down projection). Rank j is owned by four warps (one per quarter of K)
+// whose lanes take 8-element chunks; a shuffle tree and a fixed-order sum of
+// the four quarters finish it (deterministic). MT = 1: 16 CTAs of 16 warps
+// (4 ranks per CTA per pass); MT > 1: one CTA of 4 warps per rank. Kept
+// small in SMs so that the GEMV behind it fits on the GPU beside it and
+// streams its weights meanwhile. It waits for everything in front of it
+// before reading anything and only then lets the GEMV start, so the GEMV may
+// read x without waiting.
+template <int MT>
+__global__ void __launch_bounds__(MT == 1 ? 512 : 128, MT == 1 ? 2 : 1) k_lora_down_small(LoraDownSmallParams p) {
+  __shared__ float s_q[16][MT];     // per warp: partial sums of its quarter
+  grid_dependency_wait();
+  grid_dependency_trigger();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  float acc[16];
+  const int ranks_per_pass = (MT == 1) ? 4 * gridDim.x : gridDim.x;
+  const int rank_in_cta = warp >> 2;
+  const int quarter = warp & 3;
+  const int64_t nch = p.k >> 3;
+  const int64_t q0 = nch * quarter / 4, q1 = nch * (quarter + 1) / 4;
+  for (int jb = 0; jb < p.r64; jb += ranks_per_pass) {
+    const int j = jb + ((MT == 1) ? blockIdx.x * 4 + rank_in_cta : blockIdx.x);
+    float acc[MT];
 #pragma unroll
-  for (int m = 0; m < 16; ++m) acc[m] = 0.0f;
-  if (j < p.r) {
-    const int64_t nch = p.k >> 3;
-    const uint4* arow = reinterpret_cast<const uint4*>(p.a + static_cast<int64_t>(j) * p.k);
-    for (int64_t c = threadIdx.x; c < nch; c += blockDim.x) {
-      const uint4 av = __ldg(arow + c);
-      const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
-      float af[8];
+    for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
+    if (j < p.r) {
+      const uint4* arow = reinterpret_cast<const uint4*>(p.a + static_cast<int64_t>(j) * p.k);
+      constexpr int kUnroll = MT == 1 ? 4 : (MT == 8 ? 2 : 1);
+#pragma unroll kUnroll
+      for (int64_t c = q0 + lane; c < q1; c += 32) {
+        const uint4 av = __ldg(arow + c);
+        const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+        float af[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        af[2 * i] = __uint_as_float(aw[i] << 16);
-        af[2 * i + 1] = __uint_as_float(aw[i] & 0xFFFF0000u);
-      }
+        for (int i = 0; i < 4; ++i) {
+          af[2 * i] = __uint_as_float(aw[i] << 16);
+          af[2 * i + 1] = __uint_as_float(aw[i] & 0xFFFF0000u);
+        }
 #pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        if (m < p.m) {
-          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * p.k) + c);
-          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+        for (int m = 0; m < MT; ++m) {
+          if (m < p.m) {
+            const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * p.k) + c);
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            acc[m] = fmaf(af[2 * i], __uint_as_float(xw[i] << 16), acc[m]);
-            acc[m] = fmaf(af[2 * i + 1], __uint_as_float(xw[i] & 0xFFFF0000u), acc[m]);
+            for (int i = 0; i < 4; ++i) {
+              acc[m] = fmaf(af[2 * i], __uint_as_float(xw[i] << 16), acc[m]);
+              acc[m] = fmaf(af[2 * i + 1], __uint_as_float(xw[i] & 0xFFFF0000u), acc[m]);
+            }
           }
         }
       }
     }
-  }
 #pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    float v = acc[m];
+    for (int m = 0; m < MT; ++m) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    if (lane == 0) s_part[warp][m] = v;
-  }
-  __syncthreads();
-  if (threadIdx.x < p.m) {
-    const int m = threadIdx.x;
-    float v = 0.0f;
+      for (int o = 16; o > 0; o >>= 1) acc[m] += __shfl_xor_sync(0xFFFFFFFFu, acc[m], o);
+    }
+    if (lane == 0) {
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v += s_part[w][m];
-    const __nv_bfloat16 b = __float2bfloat16_rn(j < p.r ? v * p.s : 0.0f);
-    p.u_pad[static_cast<int64_t>(m) * p.r64 + j] = b;
-    if (p.u_out != nullptr && j < p.r) p.u_out[static_cast<int64_t>(m) * p.r + j] = b;
+      for (int m = 0; m < MT; ++m) s_q[warp][m] = acc[m];
+    }
+    __syncthreads();
+    // the first warp of each rank's four sums their quarters in order; lane m writes token m
+    if (quarter == 0 && lane < MT && lane < p.m && j < p.r64) {
+      const int m = lane;
+      const float v = ((s_q[warp][m] + s_q[warp + 1][m]) + s_q[warp + 2][m]) + s_q[warp + 3][m];
+      const __nv_bfloat16 b = __float2bfloat16_rn(j < p.r ? v * p.s : 0.0f);
+      p.u_pad[static_cast<int64_t>(m) * p.r64 + j] = b;
+      if (p.u_out != nullptr && j < p.r) p.u_out[static_cast<int64_t>(m) * p.r + j] = b;
+    }
+    __syncthreads();
   }
 }
+
+template __global__ void k_lora_down_small<1>(LoraDownSmallParams);
+template __global__ void k_lora_down_small<8>(LoraDownSmallParams);
+template __global__ void k_lora_down_small<16>(LoraDownSmallParams);
 
 }  // namespace qlora

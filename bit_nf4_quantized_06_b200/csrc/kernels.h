@@ -58,6 +58,7 @@ struct LoraDownSmallParams {
 
 template <int NT>
 __global__ void k_gemv_nf4(GemvParams p);
+template <int MT>
 __global__ void k_lora_down_small(LoraDownSmallParams p);
 
 // ------------------------------------------------------------ tensor-core GEMM engine

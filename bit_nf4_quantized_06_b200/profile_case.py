@@ -3,7 +3,7 @@
     python -m bit_nf4_quantized_06_b200.profile_case --op fwd --workload 7b-mlp --iters 3
 
 Ops: quantize, dequantize, fwd (tensor-core path), bwd, gemv (decode path).
-Workloads: tiny, decode, 7b-mlp, 65b-gate, 65b-down. The inputs are the
+Workloads: tiny, decode, 7b-mlp, 65b-gate, 65b-down, decode-65b-gate. The inputs are the
 seeded synthetic tensors of ``synth``; every call goes through the C ABI.
 Prints one line with the mean device time per call (CUDA events); numbers
 printed while running under a profiler are not measurements.
@@ -24,7 +24,9 @@ import synth  # noqa: E402
 import bit_nf4_quantized_06_b200 as q  # noqa: E402
 
 WORKLOADS = {"tiny": synth.TINY, "decode": synth.DECODE, "7b-mlp": synth.MLP7B,
-             "65b-gate": synth.GATE65B, "65b-down": synth.DOWN65B}
+             "65b-gate": synth.GATE65B, "65b-down": synth.DOWN65B,
+             "decode-65b-gate": synth.Problem("decode-gemv-22016x8192-m1-r64", 22016, 8192, 1, 64, 16.0,
+                                              backward=False)}
 
 
 def main(argv=None):
