@@ -11,7 +11,7 @@ Functions carry the C names:
     qlora_nf4_bytes, qlora_nf4_codebook, qlora_quantize_nf4, qlora_dequantize,
     qlora_workspace_bytes, qlora_fwd_workspace_bytes, qlora_linear_fwd, qlora_linear_fwd_ex,
     qlora_linear_fwd_noalloc, qlora_linear_bwd, qlora_device_status, qlora_status_string, qlora_version,
-    qlora_launch_count, qlora_selftest_wait_timeout
+    qlora_launch_count, qlora_selftest_wait_timeout, qlora_merge_lora, qlora_adamw_step
 """
 
 import ctypes
@@ -23,7 +23,7 @@ __all__ = [
     "qlora_workspace_bytes", "qlora_fwd_workspace_bytes", "qlora_linear_fwd", "qlora_linear_fwd_ex", "qlora_linear_fwd_noalloc",
     "qlora_linear_bwd",
     "qlora_device_status", "qlora_status_string", "qlora_version", "qlora_launch_count",
-    "qlora_selftest_wait_timeout",
+    "qlora_selftest_wait_timeout", "qlora_merge_lora", "qlora_adamw_step", "AdamwParams",
     "FWD_AUTO", "FWD_GEMM", "FWD_GEMV",
 ]
 
@@ -83,6 +83,16 @@ lib.qlora_status_string.argtypes = [ctypes.c_int]
 lib.qlora_status_string.restype = ctypes.c_char_p
 lib.qlora_version.argtypes = []
 lib.qlora_version.restype = _i32
+class AdamwParams(ctypes.Structure):
+    """qlora_adamw_t: lr, beta1, beta2, eps, weight_decay, step (1-based)."""
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int32)]
+
+
+lib.qlora_adamw_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, ctypes.POINTER(AdamwParams), _vp]
+lib.qlora_adamw_step.restype = ctypes.c_int
+lib.qlora_merge_lora.argtypes = [_P(Nf4Struct), _vp, _vp, _i32, _f32, _vp, _vp]
+lib.qlora_merge_lora.restype = ctypes.c_int
 lib.qlora_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _vp]
 lib.qlora_selftest_wait_timeout.restype = ctypes.c_int
 lib.qlora_launch_count.argtypes = []
@@ -281,3 +291,29 @@ def qlora_selftest_wait_timeout(limit_us, stream=None):
     """Launch the bounded-wait self test (a wait that nothing completes); the
     timeout shows up in the next qlora_device_status()."""
     _check(lib.qlora_selftest_wait_timeout(int(limit_us), _stream_ptr(stream)), "qlora_selftest_wait_timeout")
+
+
+def qlora_merge_lora(q, a, b, alpha, out=None, stream=None):
+    """bf16(W_hat + (alpha/r) B A) as a new [N, K] bf16 tensor (or into `out`)."""
+    torch = _torch()
+    r = a.shape[0]
+    if out is None:
+        out = torch.empty((q.n_out, q.k_in), dtype=torch.bfloat16, device=q.codes.device)
+    s = q.struct()
+    _check(lib.qlora_merge_lora(ctypes.byref(s), _ptr(a), _ptr(b), r, float(alpha), _ptr(out),
+                                _stream_ptr(stream)), "qlora_merge_lora")
+    return out
+
+
+def qlora_adamw_step(master, grad, m, v, step, lr=1e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0,
+                     param=None, stream=None):
+    """One AdamW step in place on fp32 `master`, `m`, `v` (device tensors or
+    pinned host tensors the GPU can address); `param` (bf16, optional)
+    receives the bf16 copy. All arguments hold the same number of elements."""
+    n = master.numel()
+    for t in (grad, m, v) + ((param,) if param is not None else ()):
+        if t.numel() != n:
+            raise ValueError("qlora_adamw_step: element counts differ")
+    hp = AdamwParams(float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay), int(step))
+    _check(lib.qlora_adamw_step(_ptr(master), _ptr(param) if param is not None else None, _ptr(grad), _ptr(m),
+                                _ptr(v), n, ctypes.byref(hp), _stream_ptr(stream)), "qlora_adamw_step")

@@ -161,6 +161,9 @@ qlora_status_t device_ready(int* sms_out, int* pairs_out = nullptr) {
     if (e == cudaSuccess) e = set_small_attrs<128>();
     if (e == cudaSuccess) e = set_small_attrs<192>();
     if (e == cudaSuccess) e = set_small_attrs<256>();
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_merge_lora, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(merge_smem_bytes(kMaxRank)));
     if (e != cudaSuccess) return QLORA_ERR_CUDA;
     st.attrs = true;
   }
@@ -783,6 +786,76 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
     if (s != QLORA_OK) return s;
   }
   return QLORA_OK;
+}
+
+qlora_status_t qlora_merge_lora(const qlora_nf4_t* q, const void* a, const void* b, int32_t r, float alpha,
+                                void* w_out, void* stream) {
+  qlora_status_t s = check_nf4(q);
+  if (s != QLORA_OK) return s;
+  if (r < 1 || r > kMaxRank) return QLORA_ERR_SHAPE;
+  if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  if (a == nullptr || b == nullptr || w_out == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(w_out)) return QLORA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(b) & 1u) != 0) return QLORA_ERR_ALIGNMENT;
+  int sms = 0;
+  if ((s = device_ready(&sms)) != QLORA_OK) return s;
+  MergeParams p{};
+  p.codes = q->codes;
+  p.q2 = q->scale_codes;
+  p.smax = q->absmax;
+  p.a = static_cast<const __nv_bfloat16*>(a);
+  p.b = static_cast<const __nv_bfloat16*>(b);
+  p.out = static_cast<__nv_bfloat16*>(w_out);
+  p.n = q->n_out;
+  p.k = q->k_in;
+  p.r = r;
+  p.r64 = r64_of(r);
+  p.s = alpha / static_cast<float>(r);
+  std::memcpy(p.cb, tables().cb, sizeof(p.cb));
+  const size_t smem = merge_smem_bytes(p.r64);
+  const dim3 grid(static_cast<unsigned>(cdiv(p.k, 128)), static_cast<unsigned>(cdiv(p.n, 128)), 1);
+  if (grid.y > 65535u) return QLORA_ERR_SHAPE;
+  k_merge_lora<<<grid, 256, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  return launch_status();
+}
+
+qlora_status_t qlora_adamw_step(float* master, void* param_bf16, const float* grad, float* m, float* v, int64_t n,
+                                const qlora_adamw_t* hp, void* stream) {
+  if (hp == nullptr || n < 0) return QLORA_ERR_INVALID_ARG;
+  if (n == 0) return QLORA_OK;
+  if (master == nullptr || grad == nullptr || m == nullptr || v == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (hp->step < 1 || !(hp->lr >= 0.0f) || !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) ||
+      !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) || !(hp->eps > 0.0f) || !std::isfinite(hp->weight_decay))
+    return QLORA_ERR_INVALID_ARG;
+  const auto a4 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if ((reinterpret_cast<uintptr_t>(master) | reinterpret_cast<uintptr_t>(grad) | reinterpret_cast<uintptr_t>(m) |
+       reinterpret_cast<uintptr_t>(v)) & 3u)
+    return QLORA_ERR_ALIGNMENT;
+  if (param_bf16 != nullptr && (reinterpret_cast<uintptr_t>(param_bf16) & 1u)) return QLORA_ERR_ALIGNMENT;
+  int sms = 0;
+  qlora_status_t s = device_ready(&sms);
+  if (s != QLORA_OK) return s;
+  AdamwParams a{};
+  a.master = master;
+  a.grad = grad;
+  a.m = m;
+  a.v = v;
+  a.param = static_cast<__nv_bfloat16*>(param_bf16);
+  a.n = n;
+  a.beta1 = hp->beta1;
+  a.beta2 = hp->beta2;
+  a.eps = hp->eps;
+  // step constants in double, rounded once
+  const double bc1 = 1.0 - std::pow(static_cast<double>(hp->beta1), hp->step);
+  const double bc2 = 1.0 - std::pow(static_cast<double>(hp->beta2), hp->step);
+  a.decay = static_cast<float>(1.0 - static_cast<double>(hp->lr) * hp->weight_decay);
+  a.step_size = static_cast<float>(hp->lr / bc1);
+  a.inv_sqrt_bc2 = static_cast<float>(1.0 / std::sqrt(bc2));
+  a.vec4 = a4(master) && a4(grad) && a4(m) && a4(v) &&
+           (param_bf16 == nullptr || (reinterpret_cast<uintptr_t>(param_bf16) & 7u) == 0);
+  const int blocks = static_cast<int>(std::min<int64_t>(cdiv(cdiv(n, 4), 256), int64_t(sms) * 8));
+  k_adamw<<<std::max(blocks, 1), 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return launch_status();
 }
 
 static_assert(QLORA_DEV_TIMEOUT_PRODUCER == QLORA_STATUS_BIT_PRODUCER && QLORA_DEV_TIMEOUT_MMA == QLORA_STATUS_BIT_MMA &&

@@ -156,6 +156,40 @@ __global__ void k_reduce_splits(SmallParams p);
 
 __global__ void k_selftest_wait(uint64_t limit_ns);
 
+// LoRA merge for export: out = bf16(W_hat + s B A), 128 x 128 tiles.
+struct MergeParams {
+  const uint8_t* codes;
+  const uint8_t* q2;
+  const float* smax;
+  const __nv_bfloat16* a;   // [r x K]
+  const __nv_bfloat16* b;   // [N x r]
+  __nv_bfloat16* out;       // [N x K]
+  int64_t n, k;
+  int32_t r, r64;
+  float s;
+  float cb[16];
+};
+__global__ void k_merge_lora(MergeParams p);
+
+// AdamW step over n parameters (fp32 master, grad, m, v; optional bf16 copy).
+struct AdamwParams {
+  float* master;
+  const float* grad;
+  float* m;
+  float* v;
+  __nv_bfloat16* param;     // may be null
+  int64_t n;
+  float beta1, beta2, eps;
+  float decay;              // 1 - lr * weight_decay
+  float step_size;          // lr / (1 - beta1^t)
+  float inv_sqrt_bc2;       // 1 / sqrt(1 - beta2^t)
+  int32_t vec4;             // all pointers 16-byte aligned (param 8-byte)
+};
+__global__ void k_adamw(AdamwParams a);
+inline size_t merge_smem_bytes(int r64) {
+  return static_cast<size_t>(128) * (r64 + 8) * 2 + static_cast<size_t>(r64) * 136 * 2 + 128 * 132 * 4;
+}
+
 // Zero-padded copy of a [rows x r] bf16 matrix into [rows x r64].
 __global__ void k_pad_cols(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
                            int64_t rows, int32_t r, int32_t r64);

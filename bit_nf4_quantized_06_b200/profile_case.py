@@ -2,7 +2,8 @@
 
     python -m bit_nf4_quantized_06_b200.profile_case --op fwd --workload 7b-mlp --iters 3
 
-Ops: quantize, dequantize, fwd (tensor-core path), bwd, gemv (decode path).
+Ops: quantize, dequantize, fwd (tensor-core path), bwd, gemv (decode path),
+merge (LoRA merge for export), adamw (adapter optimizer step, states on device).
 Workloads: tiny, decode, 7b-mlp, 65b-gate, 65b-down, decode-65b-gate. The inputs are the
 seeded synthetic tensors of ``synth``; every call goes through the C ABI.
 Prints one line with the mean device time per call (CUDA events); numbers
@@ -31,7 +32,7 @@ WORKLOADS = {"tiny": synth.TINY, "decode": synth.DECODE, "7b-mlp": synth.MLP7B,
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["quantize", "dequantize", "fwd", "bwd", "gemv"], required=True)
+    ap.add_argument("--op", choices=["quantize", "dequantize", "fwd", "bwd", "gemv", "merge", "adamw"], required=True)
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="7b-mlp")
     ap.add_argument("--iters", type=int, default=3)
     a = ap.parse_args(argv)
@@ -45,6 +46,10 @@ def main(argv=None):
     u = torch.empty((p.m, p.r), dtype=torch.bfloat16, device="cuda")
     q.qlora_linear_fwd_ex(qw, x, aa, bb, p.alpha, path=q.FWD_GEMM if p.m > 16 else q.FWD_GEMV, y=y, u=u, ws=ws)
     w_out = torch.empty_like(w)
+    na = aa.numel() + bb.numel()
+    master = torch.zeros(na, device="cuda")
+    grad = torch.full((na,), 1e-3, device="cuda")
+    m_st, v_st = torch.zeros(na, device="cuda"), torch.zeros(na, device="cuda")
 
     def call():
         if a.op == "quantize":
@@ -53,6 +58,10 @@ def main(argv=None):
             q.qlora_dequantize(qw, out=w_out)
         elif a.op == "fwd":
             q.qlora_linear_fwd_ex(qw, x, aa, bb, p.alpha, path=q.FWD_GEMM, y=y, u=u, ws=ws)
+        elif a.op == "merge":
+            q.qlora_merge_lora(qw, aa, bb, p.alpha, out=w_out)
+        elif a.op == "adamw":
+            q.qlora_adamw_step(master, grad, m_st, v_st, 1)
         elif a.op == "gemv":
             q.qlora_linear_fwd_ex(qw, x, aa, bb, p.alpha, path=q.FWD_GEMV, y=y, ws=ws, want_u=False)
         else:

@@ -177,6 +177,40 @@ QLORA_API qlora_status_t qlora_linear_bwd(const qlora_nf4_t *q, const void *x_bf
                                 const void *b_bf16, int32_t r, float alpha, void *dx_bf16,
                                 float *da, float *db, void *ws, size_t ws_bytes, void *stream);
 
+/* LoRA merge for export: w_out [N x K] bf16 (device, row-major, caller-owned)
+ * receives bf16(W_hat + (alpha/r) B A), with W_hat the restored weight of q
+ * (exactly what qlora_dequantize writes), the rank-r product accumulated in
+ * fp32 and one rounding to bf16 at the end. This is the export path of
+ * "48GB GPU Fine-Tuning a 65B Model: Where QLoRA Saves GPU Memory":
+ * § "LoRA Freezes the Original Weights ..." (B A has W's shape and is added
+ * to it, so inference pays nothing extra) and § "QLoRA Puts the Two Methods
+ * in Different Places" (with a 4-bit base the adapters are merged into the
+ * restored 16-bit weights, not into the codes). A [r x K] and w_out must be
+ * 16-byte aligned; B [N x r] 2-byte aligned. 1 <= r <= 256. */
+QLORA_API qlora_status_t qlora_merge_lora(const qlora_nf4_t *q, const void *a_bf16, const void *b_bf16,
+                                          int32_t r, float alpha, void *w_out_bf16, void *stream);
+
+/* AdamW step for the LoRA adapters (A and B are the only trained
+ * parameters; their Adam states m and v may live in CPU pinned memory:
+ * «QLoRA는 어떻게 65B 모델을 GPU 한 장에 올렸나», § "메모리 회계: 세 겹의 최적화",
+ * Paged Optimizer). The update runs on the GPU; `master`, `m` and `v` may be
+ * device memory or pinned host memory the GPU can address (then each step
+ * moves 16 bytes per parameter over the host link and keeps nothing of it on
+ * the device). Update, with t = step (1-based):
+ *   m <- b1 m + (1-b1) g;  v <- b2 v + (1-b2) g^2;  p <- p (1 - lr wd)
+ *   p <- p - (lr / (1-b1^t)) m / (sqrt(v) / sqrt(1-b2^t) + eps)
+ * master (fp32, n), m, v (fp32, n) are updated in place; grad (fp32, n) is
+ * read (e.g. dA or dB from qlora_linear_bwd); param_bf16 (n, may be NULL)
+ * receives bf16(master) for the next forward. All fp32 pointers 4-byte
+ * aligned (16-byte aligned ones take the vector path). Asynchronous on
+ * `stream`: launch it on a second stream to overlap it with other work. */
+typedef struct {
+  float lr, beta1, beta2, eps, weight_decay;
+  int32_t step;
+} qlora_adamw_t;
+QLORA_API qlora_status_t qlora_adamw_step(float *master, void *param_bf16, const float *grad, float *m,
+                                          float *v, int64_t n, const qlora_adamw_t *hp, void *stream);
+
 /* Synchronises `stream`, then reads and clears the device status word of the
  * current device. Returns QLORA_OK, QLORA_ERR_TIMEOUT (a kernel gave up on a
  * bounded wait; *bits, if non-NULL, gets which role), or QLORA_ERR_CUDA. */

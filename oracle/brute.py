@@ -10,7 +10,10 @@ checked against them:
   Reduces Bits per Number");
 * the forward and backward are explicit triple loops of the formulas in
   «QLoRA는 어떻게 65B 모델을 GPU 한 장에 올렸나», § "QLoRA의 수식" and
-  § "명제 1".
+  § "명제 1";
+* the merge for export adds s B A to the restored weight and rounds the
+  exact sum once to bf16 ("48GB GPU Fine-Tuning a 65B Model ...",
+  § "QLoRA Puts the Two Methods in Different Places").
 
 Float32 divisions are evaluated exactly with ``fractions.Fraction`` and
 rounded once to binary32 (ties to even), so no numpy or float64
@@ -131,3 +134,51 @@ def forward(x, w_hat, a, b, s):
             row.append(base[m][n] + s * lora)
         y.append(row)
     return y
+
+
+def bf16_round_bits(q):
+    """Round an exact rational to the nearest bfloat16 (ties to even); uint16 bits."""
+    q = Fraction(q)
+    if q == 0:
+        return 0
+    sign = 0x8000 if q < 0 else 0
+    q = abs(q)
+    e = q.numerator.bit_length() - q.denominator.bit_length()
+    if Fraction(2) ** e > q:
+        e -= 1
+    if Fraction(2) ** (e + 1) <= q:
+        e += 1
+    e = max(e, -126)
+    ulp = Fraction(2) ** (e - 7)          # 8 significant bits
+    n = q / ulp
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    val = fl * ulp                        # exact, representable (or the next binade)
+    if val == 0:
+        return sign
+    ee = val.numerator.bit_length() - val.denominator.bit_length()
+    if Fraction(2) ** ee > val:
+        ee -= 1
+    if ee < -126:                         # subnormal: exponent field 0
+        frac = int(val / Fraction(2) ** -133)
+        return sign | frac
+    frac = int((val / Fraction(2) ** ee - 1) * 128)
+    return sign | ((ee + 127) << 7) | frac
+
+
+def merge(w_hat, a, b, s):
+    """bf16 bits of W_hat[n][k] + s * sum_j B[n][j] A[j][k], summed exactly, one rounding."""
+    n, k, r = len(w_hat), len(w_hat[0]), len(a)
+    sf = Fraction(s)
+    out = []
+    for i in range(n):
+        row = []
+        for c in range(k):
+            acc = Fraction(0)
+            for j in range(r):
+                acc += Fraction(b[i][j]) * Fraction(a[j][c])
+            row.append(bf16_round_bits(Fraction(w_hat[i][c]) + sf * acc))
+        out.append(row)
+    return out

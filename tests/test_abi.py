@@ -87,3 +87,26 @@ def test_argument_validation_before_any_launch(q):
     s = q.Nf4Struct(512, 512, 64, 256, 17, 16, 16)       # misaligned codes
     assert lib.qlora_dequantize(ctypes.byref(s), ctypes.c_void_p(16), None) == 3
     assert lib.qlora_nf4_codebook(None) == 1
+
+
+def test_merge_argument_validation(q):
+    lib = q.lib
+    s = q.Nf4Struct(512, 512, 64, 256, 16, 16, 16)
+    assert lib.qlora_merge_lora(ctypes.byref(s), ctypes.c_void_p(16), ctypes.c_void_p(16), 0, 16.0,
+                                ctypes.c_void_p(16), None) == 2      # r out of range
+    assert lib.qlora_merge_lora(ctypes.byref(s), None, ctypes.c_void_p(16), 8, 16.0,
+                                ctypes.c_void_p(16), None) == 1      # null A
+    assert lib.qlora_merge_lora(ctypes.byref(s), ctypes.c_void_p(24), ctypes.c_void_p(16), 8, 16.0,
+                                ctypes.c_void_p(16), None) == 3      # misaligned A
+
+
+def test_adamw_argument_validation(q):
+    lib = q.lib
+    hp = q.AdamwParams(1e-3, 0.9, 0.999, 1e-8, 0.0, 0)                 # step must be >= 1
+    f = ctypes.c_void_p(16)
+    assert lib.qlora_adamw_step(f, None, f, f, f, 10, ctypes.byref(hp), None) == 1
+    hp.step = 1
+    assert lib.qlora_adamw_step(ctypes.c_void_p(18), None, f, f, f, 10, ctypes.byref(hp), None) == 3
+    assert lib.qlora_adamw_step(f, None, f, f, f, 0, ctypes.byref(hp), None) == 0   # nothing to do
+    hp.beta1 = 1.0
+    assert lib.qlora_adamw_step(f, None, f, f, f, 10, ctypes.byref(hp), None) == 1

@@ -1,0 +1,88 @@
+"""GPU parity of the LoRA merge for export (bf16(W_hat + s B A)).
+
+The oracle forms the sum exactly (float64) and rounds once to bf16; the GPU
+accumulates B A in fp32 on the tensor cores, multiplies by s in fp32, adds
+the exactly restored weight in fp32 and rounds once. The two can differ only
+where the fp32 path lands on the other side of a bf16 rounding boundary, by
+one unit in the last place: the test requires that bound everywhere and
+bit equality for all but a tiny fraction of the weights.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import linear, nf4
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    import bit_nf4_quantized_06_b200 as q
+    return q
+
+
+def _ulps(a_bits, b_bits):
+    # distance in bf16 steps between two arrays of bf16 bit patterns (same sign side)
+    def key(b):
+        b = b.astype(np.int32)
+        return np.where(b & 0x8000, -(b & 0x7FFF), b)
+    return np.abs(key(a_bits) - key(b_bits))
+
+
+CASES = [
+    # n, k, r, alpha, outliers, b_scale
+    (256, 256, 8, 16.0, False, 1.0),
+    (200, 192, 12, 16.0, False, 30.0),     # ragged rows and k-tiles, r not a multiple of 8, visible adapter
+    (384, 1024, 100, 32.0, True, 10.0),
+    (128, 512, 256, 16.0, False, 5.0),     # largest rank
+]
+
+
+@pytest.mark.parametrize("n,k,r,alpha,outl,bs", CASES)
+def test_merge_parity(q, n, k, r, alpha, outl, bs):
+    w = synth.weight(n, k, seed=n + k, outliers=outl)
+    a = synth.lora_a(r, k, seed=3)
+    b = (synth.lora_b(n, r, seed=4).float() * bs).to(torch.bfloat16)
+    o = nf4.quantize(w.float().numpy())
+    w_hat = nf4.dequantize(o["codes"], o["q2"], o["smax"])
+    ref = linear.merge_bits(w_hat, a.float().numpy(), b.float().numpy(), np.float32(alpha) / np.float32(r))
+    qw = q.qlora_quantize_nf4(w.cuda())
+    got = q.qlora_merge_lora(qw, a.cuda(), b.cuda(), alpha)
+    torch.cuda.synchronize()
+    gb = got.cpu().view(torch.int16).numpy().view(np.uint16)
+    d = _ulps(gb, ref)
+    assert d.max() <= 1
+    assert np.mean(d != 0) < 1e-3
+    assert q.qlora_device_status() == (0, 0)
+
+
+def test_merge_b_zero_is_restore(q):
+    n, k, r = 320, 448, 16
+    w = synth.weight(n, k, seed=8)
+    qw = q.qlora_quantize_nf4(w.cuda())
+    a = synth.lora_a(r, k).cuda()
+    b = torch.zeros((n, r), dtype=torch.bfloat16, device="cuda")
+    got = q.qlora_merge_lora(qw, a, b, 16.0)
+    w_hat = q.qlora_dequantize(qw)
+    torch.cuda.synchronize()
+    assert torch.equal(got.view(torch.int16), w_hat.view(torch.int16))
+
+
+def test_merge_full_size_7b_mlp(q):
+    p = synth.MLP7B
+    w = synth.weight(p.n, p.k)
+    a = synth.lora_a(p.r, p.k)
+    b = (synth.lora_b(p.n, p.r).float() * 10.0).to(torch.bfloat16)
+    o = nf4.quantize(w.float().numpy())
+    w_hat = nf4.dequantize(o["codes"], o["q2"], o["smax"])
+    rows = np.array([0, 1, 127, 128, 5000, 11007])
+    ref = linear.merge_bits(w_hat[rows], a.float().numpy(), b.float().numpy()[rows], np.float32(p.scale))
+    qw = q.qlora_quantize_nf4(w.cuda())
+    got = q.qlora_merge_lora(qw, a.cuda(), b.cuda(), p.alpha)
+    torch.cuda.synchronize()
+    gb = got.cpu().view(torch.int16).numpy().view(np.uint16)[rows]
+    d = _ulps(gb, ref)
+    assert d.max() <= 1 and np.mean(d != 0) < 1e-3

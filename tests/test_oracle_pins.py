@@ -17,7 +17,7 @@ import pytest
 import torch
 
 import synth
-from oracle import bf16, brute, linear, nf4
+from oracle import bf16, brute, linear, nf4, optim
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -329,3 +329,80 @@ def test_backward_has_no_weight_gradient_and_b_zero():
 def test_rel_fro():
     a = np.array([3.0, 4.0])
     assert linear.rel_fro(a * 1.01, a) == pytest.approx(0.01)
+
+
+# --------------------------------------------------------------------------- merge for export
+
+def test_merge_matches_exact_rational_loops():
+    # exact rational sum, one rounding to bf16, against the vectorised oracle
+    for s in (4.0, 16.0 / 12.0, -0.375):
+        x, w, a, b, _ = _small(n=6, k=64, r=5, seed=21)
+        got = linear.merge_bits(w, a, b, s)
+        ref = np.array(brute.merge(w.tolist(), a.tolist(), b.tolist(), s), dtype=np.uint16)
+        assert np.array_equal(got, ref)
+
+
+def test_merge_rounding_at_bf16_ties():
+    # W_hat + s B A placed exactly on, and one float64 step either side of,
+    # bf16 rounding ties: the oracle must follow round-to-nearest-even there
+    w = np.array([[1.0, 1.0, 1.0, 1.0]], dtype=np.float32)
+    half_ulp = 2.0 ** -8                  # bf16 spacing at 1.0 is 2^-7
+    a = np.array([[half_ulp, 3 * half_ulp, half_ulp + 2.0 ** -40, half_ulp - 2.0 ** -40]])
+    b = np.array([[1.0]])
+    got = linear.merge_bits(w, a, b, 1.0)
+    ref = np.array(brute.merge(w.tolist(), a.tolist(), b.tolist(), 1.0), dtype=np.uint16)
+    assert np.array_equal(got, ref)
+    # 1 + 2^-8 ties to 1.0 (even); 1 + 3*2^-8 ties to 1 + 2^-6 (even); off-tie values go to the nearer side
+    assert got[0, 0] == 0x3F80 and got[0, 1] == 0x3F82 and got[0, 2] == 0x3F81 and got[0, 3] == 0x3F80
+
+
+def test_merge_with_b_zero_is_restored_weight():
+    w = synth.weight(64, 128, seed=4).float().numpy()
+    o = nf4.quantize(w)
+    w_hat = nf4.dequantize(o["codes"], o["q2"], o["smax"])
+    a = synth.lora_a(8, 128).float().numpy()
+    got = linear.merge_bits(w_hat, a, np.zeros((64, 8)), 2.0)
+    assert np.array_equal(got, nf4.dequantize_bits(o["codes"], o["q2"], o["smax"]))
+
+
+def test_merged_forward_matches_adapter_forward():
+    # the merged model's forward equals the base + adapter forward up to the
+    # bf16 rounding of the merged weight
+    t = synth.make(synth.TINY)
+    o = nf4.quantize(t["w"].float().numpy())
+    w_hat = nf4.dequantize(o["codes"], o["q2"], o["smax"])
+    x, a, b = (t[k_].float().numpy() for k_ in ("x", "a", "b"))
+    b = b * 50.0                          # make the adapter term visible next to W_hat
+    s = synth.TINY.scale
+    merged = bf16.bf16_bits_to_f32(linear.merge_bits(w_hat, a, b, s))
+    y_ref, _ = linear.forward(x, w_hat, a, b, s)
+    y_m = x.astype(np.float64) @ merged.astype(np.float64).T
+    assert linear.rel_fro(y_m, y_ref) <= 2.0 ** -8
+    assert linear.rel_fro(y_m, x.astype(np.float64) @ w_hat.astype(np.float64).T) > 1e-2
+
+
+# --------------------------------------------------------------------------- AdamW for the adapters
+
+def test_adamw_first_step_closed_form():
+    # t = 1, wd = 0: m_hat = g and v_hat = g^2, so the step is lr * g / (|g| + eps)
+    g = np.array([0.5, -2.0, 1e-3, 0.0, -7.25])
+    p0 = np.array([1.0, -1.0, 0.5, 0.25, 3.0])
+    p1, m1, v1 = optim.adamw_step(p0, g, np.zeros(5), np.zeros(5), 1, 1e-3, 0.9, 0.999, 1e-8, 0.0)
+    assert np.allclose(p1, p0 - 1e-3 * g / (np.abs(g) + 1e-8), rtol=1e-14, atol=1e-15)
+    assert np.allclose(m1, 0.1 * g) and np.allclose(v1, 0.001 * g * g)
+
+
+def test_adamw_matches_torch_adamw():
+    # the update rule equals the library's AdamW (float64) over several steps
+    rng = np.random.default_rng(3)
+    p = rng.standard_normal(300)
+    m = np.zeros(300)
+    v = np.zeros(300)
+    tp = torch.tensor(p.copy(), dtype=torch.float64, requires_grad=True)
+    opt = torch.optim.AdamW([tp], lr=2e-3, betas=(0.9, 0.995), eps=1e-7, weight_decay=0.05)
+    for t in range(1, 6):
+        g = rng.standard_normal(300)
+        p, m, v = optim.adamw_step(p, g, m, v, t, 2e-3, 0.9, 0.995, 1e-7, 0.05)
+        tp.grad = torch.tensor(g, dtype=torch.float64)
+        opt.step()
+    assert np.allclose(p, tp.detach().numpy(), rtol=1e-13, atol=1e-15)
