@@ -325,11 +325,14 @@ def merge_timing(q, wl, l2, reps=10):
 
 
 def paged_optimizer(q, wl, l2, reps=10):
-    """AdamW for one adapter pair (A: r x K, B: N x r) with m, v in pinned host
-    memory: standalone time (host states vs device states) and the cost of
-    running it on a second stream beside a step's backward (the update of the
-    layer before, as in a stack where layer L's update overlaps layer L-1's
-    backward)."""
+    """AdamW for one adapter pair (A: r x K, B: N x r, 966,656 parameters at
+    the 7B-MLP shape) with m, v paged out to pinned host memory, two ways:
+    the GPU kernel reading the host states over the link, and the pages' own
+    scheme (gradient copied to the host, update on the CPU as a host function
+    of a side stream, bf16 adapter copied back). Each is timed alone and as
+    the update of "the layer before" running on a second stream beside a
+    step's backward (as in a stack, where layer L's update overlaps layer
+    L-1's backward); the loss is the step time it adds."""
     p, dev = wl.p, wl.x.device
     n = p.r * p.k + p.n * p.r
     hp = dict(lr=1e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0)
@@ -338,51 +341,74 @@ def paged_optimizer(q, wl, l2, reps=10):
     grad = torch.randn(n, device=dev) * 1e-3
     m_h, v_h = torch.zeros(n).pin_memory(), torch.zeros(n).pin_memory()
     m_d, v_d = torch.zeros(n, device=dev), torch.zeros(n, device=dev)
+    master_h = (torch.randn(n) * 0.01).pin_memory()
+    grad_h = torch.empty(n).pin_memory()
+    param_h = torch.empty(n, dtype=torch.bfloat16).pin_memory()
+    side = torch.cuda.Stream(device=dev)
 
-    def timed(m, v):
+    def gpu_host_states(i, stream=None):
+        q.qlora_adamw_step(master, grad, m_h, v_h, i + 1, param=param, stream=stream, **hp)
+
+    def gpu_device_states(i, stream=None):
+        q.qlora_adamw_step(master, grad, m_d, v_d, i + 1, param=param, stream=stream, **hp)
+
+    def cpu_paged(i, stream=None):
+        q.qlora_adamw_paged(grad, master_h, m_h, v_h, grad_h, i + 1, param_dev=param, param_host=param_h,
+                            stream=stream, **hp)
+
+    def alone(fn):
         ts = []
         for i in range(reps):
             flush_l2(l2)
+            torch.cuda.synchronize()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            q.qlora_adamw_step(master, grad, m, v, i + 1, param=param, **hp)
+            fn(i)
             e1.record()
             torch.cuda.synchronize()
             ts.append(e0.elapsed_time(e1))
         return float(np.median(ts))
 
-    t_host = timed(m_h, v_h)
-    t_dev = timed(m_d, v_d)
-    # overlap: the step on the main stream, the update on a side stream started with the backward
-    side = torch.cuda.Stream(device=dev)
-    base, over = [], []
-    for i in range(reps):
-        for with_opt in (False, True):
-            flush_l2(l2)
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            eb = torch.cuda.Event()
-            e0.record()
-            q.qlora_quantize_nf4(wl.w, out=wl.qw)
-            q.qlora_linear_fwd(wl.qw, wl.x, wl.a, wl.b, p.alpha, y=wl.y, u=wl.u, ws=wl.ws)
-            eb.record()
-            if with_opt:
-                side.wait_event(eb)
-                q.qlora_adamw_step(master, grad, m_h, v_h, i + 1, param=param, stream=side, **hp)
-            q.qlora_linear_bwd(wl.qw, wl.x, wl.u, wl.dy, wl.a, wl.b, p.alpha, dx=wl.dx, da=wl.da, db=wl.db,
-                               ws=wl.ws)
-            if with_opt:
-                torch.cuda.current_stream().wait_stream(side)
-            e1.record()
-            torch.cuda.synchronize()
-            (over if with_opt else base).append(e0.elapsed_time(e1))
-    tb, to = float(np.median(base)), float(np.median(over))
-    return {"params": n, "ms_host_states": round(t_host, 4), "ms_device_states": round(t_dev, 4),
-            "host_link_GB/s": round(16.0 * n / (t_host * 1e-3) / 1e9, 1),
-            "step_ms": round(tb, 4), "step_ms_with_paged_update": round(to, 4),
-            "throughput_loss": round(to / tb - 1.0, 4),
-            "method": "7B-MLP quantize+fwd+bwd with an adapter AdamW (states in pinned host memory) on a "
-                      "second stream from the start of the backward; medians of 10"}
+    def beside_step(fn):
+        base, over = [], []
+        for i in range(reps):
+            for with_opt in (False, True):
+                flush_l2(l2)
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                eb = torch.cuda.Event()
+                e0.record()
+                q.qlora_quantize_nf4(wl.w, out=wl.qw)
+                q.qlora_linear_fwd(wl.qw, wl.x, wl.a, wl.b, p.alpha, y=wl.y, u=wl.u, ws=wl.ws)
+                eb.record()
+                if with_opt:
+                    side.wait_event(eb)
+                    fn(i, stream=side)
+                q.qlora_linear_bwd(wl.qw, wl.x, wl.u, wl.dy, wl.a, wl.b, p.alpha, dx=wl.dx, da=wl.da, db=wl.db,
+                                   ws=wl.ws)
+                if with_opt:
+                    torch.cuda.current_stream().wait_stream(side)
+                e1.record()
+                torch.cuda.synchronize()
+                (over if with_opt else base).append(e0.elapsed_time(e1))
+        tb, to = float(np.median(base)), float(np.median(over))
+        return tb, to
+
+    t_dev = alone(gpu_device_states)
+    t_hostk = alone(gpu_host_states)
+    t_cpu = alone(cpu_paged)
+    tb1, to1 = beside_step(gpu_host_states)
+    tb2, to2 = beside_step(cpu_paged)
+    return {"params": n,
+            "ms_device_states": round(t_dev, 4),
+            "gpu_update_host_states": {"ms": round(t_hostk, 4), "host_link_GB/s": round(16.0 * n / (t_hostk * 1e-3) / 1e9, 1),
+                                       "step_ms": round(tb1, 4), "step_ms_with_update": round(to1, 4),
+                                       "throughput_loss": round(to1 / tb1 - 1.0, 4)},
+            "cpu_update_paged": {"ms": round(t_cpu, 4), "cpu_threads": os.cpu_count(),
+                                 "step_ms": round(tb2, 4), "step_ms_with_update": round(to2, 4),
+                                 "throughput_loss": round(to2 / tb2 - 1.0, 4)},
+            "method": "7B-MLP quantize+fwd+bwd on the main stream; the update on a second stream from the start "
+                      "of the backward; medians of 10"}
 
 
 def cpu_baseline_sample(target_s=15.0):

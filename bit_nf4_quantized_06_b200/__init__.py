@@ -11,7 +11,8 @@ Functions carry the C names:
     qlora_nf4_bytes, qlora_nf4_codebook, qlora_quantize_nf4, qlora_dequantize,
     qlora_workspace_bytes, qlora_fwd_workspace_bytes, qlora_linear_fwd, qlora_linear_fwd_ex,
     qlora_linear_fwd_noalloc, qlora_linear_bwd, qlora_device_status, qlora_status_string, qlora_version,
-    qlora_launch_count, qlora_selftest_wait_timeout, qlora_merge_lora, qlora_adamw_step
+    qlora_launch_count, qlora_selftest_wait_timeout, qlora_merge_lora, qlora_adamw_step, qlora_adamw_host,
+    qlora_adamw_paged
 """
 
 import ctypes
@@ -23,7 +24,8 @@ __all__ = [
     "qlora_workspace_bytes", "qlora_fwd_workspace_bytes", "qlora_linear_fwd", "qlora_linear_fwd_ex", "qlora_linear_fwd_noalloc",
     "qlora_linear_bwd",
     "qlora_device_status", "qlora_status_string", "qlora_version", "qlora_launch_count",
-    "qlora_selftest_wait_timeout", "qlora_merge_lora", "qlora_adamw_step", "AdamwParams",
+    "qlora_selftest_wait_timeout", "qlora_merge_lora", "qlora_adamw_step", "qlora_adamw_host", "qlora_adamw_paged",
+    "AdamwParams",
     "FWD_AUTO", "FWD_GEMM", "FWD_GEMV",
 ]
 
@@ -91,6 +93,10 @@ class AdamwParams(ctypes.Structure):
 
 lib.qlora_adamw_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, ctypes.POINTER(AdamwParams), _vp]
 lib.qlora_adamw_step.restype = ctypes.c_int
+lib.qlora_adamw_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, ctypes.POINTER(AdamwParams)]
+lib.qlora_adamw_host.restype = ctypes.c_int
+lib.qlora_adamw_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, ctypes.POINTER(AdamwParams), _vp]
+lib.qlora_adamw_paged.restype = ctypes.c_int
 lib.qlora_merge_lora.argtypes = [_P(Nf4Struct), _vp, _vp, _i32, _f32, _vp, _vp]
 lib.qlora_merge_lora.restype = ctypes.c_int
 lib.qlora_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _vp]
@@ -317,3 +323,24 @@ def qlora_adamw_step(master, grad, m, v, step, lr=1e-4, betas=(0.9, 0.999), eps=
     hp = AdamwParams(float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay), int(step))
     _check(lib.qlora_adamw_step(_ptr(master), _ptr(param) if param is not None else None, _ptr(grad), _ptr(m),
                                 _ptr(v), n, ctypes.byref(hp), _stream_ptr(stream)), "qlora_adamw_step")
+
+
+def qlora_adamw_host(master, grad, m, v, step, lr=1e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0,
+                     param=None):
+    """AdamW on the host CPU, in place on CPU fp32 tensors; `param` (CPU
+    bf16 tensor, optional) receives the bf16 copy."""
+    n = master.numel()
+    hp = AdamwParams(float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay), int(step))
+    _check(lib.qlora_adamw_host(_ptr(master), _ptr(param) if param is not None else None, _ptr(grad), _ptr(m),
+                                _ptr(v), n, ctypes.byref(hp)), "qlora_adamw_host")
+
+
+def qlora_adamw_paged(grad_dev, master_host, m_host, v_host, grad_host, step, param_dev=None, param_host=None,
+                      lr=1e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0, stream=None):
+    """Enqueue one paged optimizer step on `stream` (D2H grad, CPU AdamW as a
+    stream host function, H2D bf16 adapter). Host tensors must be pinned."""
+    n = master_host.numel()
+    hp = AdamwParams(float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay), int(step))
+    _check(lib.qlora_adamw_paged(_ptr(grad_dev), _ptr(param_dev), _ptr(master_host), _ptr(m_host), _ptr(v_host),
+                                 _ptr(grad_host), _ptr(param_host), n, ctypes.byref(hp), _stream_ptr(stream)),
+           "qlora_adamw_paged")

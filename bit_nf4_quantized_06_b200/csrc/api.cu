@@ -796,7 +796,8 @@ qlora_status_t qlora_merge_lora(const qlora_nf4_t* q, const void* a, const void*
   if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
   if (a == nullptr || b == nullptr || w_out == nullptr) return QLORA_ERR_INVALID_ARG;
   if (!aligned16(a) || !aligned16(w_out)) return QLORA_ERR_ALIGNMENT;
-  if ((reinterpret_cast<uintptr_t>(b) & 1u) != 0) return QLORA_ERR_ALIGNMENT;
+  // B is read 16 bytes at a time when r % 8 == 0, else element by element
+  if ((reinterpret_cast<uintptr_t>(b) & ((r % 8 == 0) ? 15u : 1u)) != 0) return QLORA_ERR_ALIGNMENT;
   int sms = 0;
   if ((s = device_ready(&sms)) != QLORA_OK) return s;
   MergeParams p{};

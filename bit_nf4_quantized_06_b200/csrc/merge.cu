@@ -95,20 +95,61 @@ __global__ void __launch_bounds__(256, 2) k_merge_lora(MergeParams p) {
     }
   }
 
-  // 1. stage B rows n0.. (r64 columns, zero past r and N) and A columns k0.. (zero past r and K)
-  for (int row = warp; row < 128; row += 8) {
-    const bool rv = n0 + row < p.n;
-    for (int j = lane; j < r64; j += 32) {
-      __nv_bfloat16 v = __float2bfloat16_rn(0.0f);
-      if (rv && j < p.r) v = p.b[(n0 + row) * p.r + j];
-      sB[row * ldb + j] = v;
+  // 1. stage B rows n0.. (r64 columns, zero past r and N) and A columns k0..
+  //    (zero past r and K); loads are issued in batches of four before their
+  //    stores so that several are in flight per thread
+  const int cpr = r64 / 8;                        // 16-byte chunks per staged B row
+  if ((p.r & 7) == 0) {
+    for (int i0 = tid; i0 < 128 * cpr; i0 += 4 * 256) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * 256;
+        const int row = i / cpr, c8 = i - row * cpr;
+        v[u] = make_uint4(0, 0, 0, 0);
+        if (i < 128 * cpr && n0 + row < p.n && c8 * 8 < p.r)
+          v[u] = __ldg(reinterpret_cast<const uint4*>(p.b + (n0 + row) * p.r + c8 * 8));
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * 256;
+        const int row = i / cpr, c8 = i - row * cpr;
+        if (i < 128 * cpr) *reinterpret_cast<uint4*>(sB + row * ldb + c8 * 8) = v[u];
+      }
+    }
+  } else {
+    for (int i0 = tid; i0 < 128 * r64; i0 += 8 * 256) {
+      __nv_bfloat16 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * 256;
+        const int row = i / r64, j = i - row * r64;
+        v[u] = __float2bfloat16_rn(0.0f);
+        if (i < 128 * r64 && n0 + row < p.n && j < p.r) v[u] = p.b[(n0 + row) * p.r + j];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * 256;
+        const int row = i / r64, j = i - row * r64;
+        if (i < 128 * r64) sB[row * ldb + j] = v[u];
+      }
     }
   }
-  for (int i = tid; i < r64 * 16; i += 256) {
-    const int j = i >> 4, c8 = i & 15;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (j < p.r && k0 + c8 * 8 < p.k) v = __ldg(reinterpret_cast<const uint4*>(p.a + j * p.k + k0 + c8 * 8));
-    *reinterpret_cast<uint4*>(sA + j * LDA + c8 * 8) = v;
+  for (int i0 = tid; i0 < r64 * 16; i0 += 4 * 256) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * 256;
+      const int j = i >> 4, c8 = i & 15;
+      v[u] = make_uint4(0, 0, 0, 0);
+      if (i < r64 * 16 && j < p.r && k0 + c8 * 8 < p.k)
+        v[u] = __ldg(reinterpret_cast<const uint4*>(p.a + j * p.k + k0 + c8 * 8));
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * 256;
+      if (i < r64 * 16) *reinterpret_cast<uint4*>(sA + (i >> 4) * LDA + (i & 15) * 8) = v[u];
+    }
   }
   __syncthreads();
 

@@ -186,7 +186,8 @@ QLORA_API qlora_status_t qlora_linear_bwd(const qlora_nf4_t *q, const void *x_bf
  * to it, so inference pays nothing extra) and § "QLoRA Puts the Two Methods
  * in Different Places" (with a 4-bit base the adapters are merged into the
  * restored 16-bit weights, not into the codes). A [r x K] and w_out must be
- * 16-byte aligned; B [N x r] 2-byte aligned. 1 <= r <= 256. */
+ * 16-byte aligned; B [N x r] 16-byte aligned when r % 8 == 0, else 2-byte
+ * aligned. 1 <= r <= 256. */
 QLORA_API qlora_status_t qlora_merge_lora(const qlora_nf4_t *q, const void *a_bf16, const void *b_bf16,
                                           int32_t r, float alpha, void *w_out_bf16, void *stream);
 
@@ -210,6 +211,27 @@ typedef struct {
 } qlora_adamw_t;
 QLORA_API qlora_status_t qlora_adamw_step(float *master, void *param_bf16, const float *grad, float *m,
                                           float *v, int64_t n, const qlora_adamw_t *hp, void *stream);
+
+/* The same update on the host CPU (the page's paged optimizer: states in
+ * CPU pinned memory, update on the CPU). All pointers are host memory;
+ * param_bf16 (may be NULL) receives bf16(master) as uint16 bit patterns.
+ * Synchronous; runs on a fixed pool of worker threads owned by the library.
+ * Never touches the GPU. */
+QLORA_API qlora_status_t qlora_adamw_host(float *master, void *param_bf16, const float *grad, float *m,
+                                          float *v, int64_t n, const qlora_adamw_t *hp);
+
+/* One paged optimizer step, enqueued on `stream` and fully asynchronous:
+ * copy grad_dev (device, n fp32) to grad_host (pinned), run
+ * qlora_adamw_host on the pinned master/m/v as a host function of the
+ * stream, then copy param_host_bf16 (pinned, n bf16) to param_dev_bf16
+ * (device; both NULL to skip). Issue it on a second stream once the
+ * gradient is complete (cudaStreamWaitEvent) so that the copies and the CPU
+ * update overlap the GPU's other work. All host buffers stay owned by the
+ * caller and must outlive the step. */
+QLORA_API qlora_status_t qlora_adamw_paged(const float *grad_dev, void *param_dev_bf16, float *master_host,
+                                           float *m_host, float *v_host, float *grad_host,
+                                           void *param_host_bf16, int64_t n, const qlora_adamw_t *hp,
+                                           void *stream);
 
 /* Synchronises `stream`, then reads and clears the device status word of the
  * current device. Returns QLORA_OK, QLORA_ERR_TIMEOUT (a kernel gave up on a

@@ -11,6 +11,12 @@ from oracle import bf16, optim
 
 pytestmark = pytest.mark.gpu
 
+def _hp32():
+    # the C ABI carries the hyperparameters as fp32: the oracle takes the same values
+    f = lambda x: float(np.float32(x))
+    return f(HP["lr"]), f(HP["betas"][0]), f(HP["betas"][1]), f(HP["eps"]), f(HP["weight_decay"])
+
+
 HP = dict(lr=2e-3, betas=(0.9, 0.995), eps=1e-8, weight_decay=0.01)
 
 
@@ -33,8 +39,7 @@ def test_adamw_parity(q, n, offset, paged):
         grad = torch.randn(n + offset, generator=g) * 0.01
         q.qlora_adamw_step(master[offset:], grad[offset:].cuda(), m[offset:], v[offset:], t, param=param[offset:], **HP)
         torch.cuda.synchronize()
-        po, mo, vo = optim.adamw_step(po, grad[offset:].double().numpy(), mo, vo, t, HP["lr"], HP["betas"][0],
-                                      HP["betas"][1], HP["eps"], HP["weight_decay"])
+        po, mo, vo = optim.adamw_step(po, grad[offset:].double().numpy(), mo, vo, t, *_hp32())
         got = master[offset:].cpu().double().numpy()
         # fp32 state against the float64 oracle: where m cancels to near zero
         # its absolute rounding (~1e-10) is amplified by step_size / denom, so
@@ -47,3 +52,26 @@ def test_adamw_parity(q, n, offset, paged):
         rb = bf16.round_f32_to_bf16_bits(master[offset:].cpu().numpy())
         assert np.array_equal(param[offset:].cpu().view(torch.int16).numpy().view(np.uint16), rb)
     assert q.qlora_device_status() == (0, 0)
+
+
+def test_paged_chain_matches_oracle(q):
+    # D2H gradient, CPU update on pinned states as a stream host function, H2D bf16 adapter
+    n = 300_001
+    g = torch.Generator().manual_seed(11)
+    master_h = (torch.randn(n, generator=g) * 0.02).pin_memory()
+    m_h, v_h = torch.zeros(n).pin_memory(), torch.zeros(n).pin_memory()
+    grad_h = torch.empty(n).pin_memory()
+    param_h = torch.empty(n, dtype=torch.bfloat16).pin_memory()
+    param_d = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    po, mo, vo = master_h.double().numpy().copy(), np.zeros(n), np.zeros(n)
+    side = torch.cuda.Stream()
+    for t in range(1, 4):
+        grad_d = (torch.randn(n, generator=g) * 0.01).cuda()
+        side.wait_stream(torch.cuda.current_stream())
+        q.qlora_adamw_paged(grad_d, master_h, m_h, v_h, grad_h, t, param_dev=param_d, param_host=param_h,
+                            stream=side, **HP)
+        side.synchronize()
+        po, mo, vo = optim.adamw_step(po, grad_d.cpu().double().numpy(), mo, vo, t, *_hp32())
+        assert np.allclose(master_h.double().numpy(), po, rtol=1e-6, atol=1e-5 * HP["lr"])
+        rb = bf16.round_f32_to_bf16_bits(master_h.numpy())
+        assert np.array_equal(param_d.cpu().view(torch.int16).numpy().view(np.uint16), rb)
