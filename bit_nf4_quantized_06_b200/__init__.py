@@ -163,28 +163,33 @@ def qlora_nf4_codebook():
 
 
 class NF4Weight:
-    """Device buffers of one packed NF4 weight (codes, scale codes, s_max)."""
+    """Device buffers of one packed NF4 weight. dq=True: codes, 8-bit scale
+    codes and one s_max per 256 blocks (double quantization); dq=False:
+    codes and one fp32 scale per 64-weight block (no scale codes)."""
 
-    def __init__(self, n_out, k_in, device="cuda"):
+    def __init__(self, n_out, k_in, device="cuda", dq=True):
         torch = _torch()
-        b_codes, b_q2, b_smax = qlora_nf4_bytes(n_out, k_in)
+        self.dq = bool(dq)
+        b_codes, b_q2, b_smax = qlora_nf4_bytes(n_out, k_in, 256 if self.dq else 0)
         self.n_out, self.k_in = int(n_out), int(k_in)
         self.codes = torch.empty(b_codes, dtype=torch.uint8, device=device)
         self.scale_codes = torch.empty(b_q2, dtype=torch.uint8, device=device)
         self.absmax = torch.empty(b_smax // 4, dtype=torch.float32, device=device)
 
     def struct(self):
-        return Nf4Struct(self.n_out, self.k_in, 64, 256, self.codes.data_ptr(), self.scale_codes.data_ptr(),
+        q2 = self.scale_codes.data_ptr() if self.dq else 0
+        return Nf4Struct(self.n_out, self.k_in, 64, 256 if self.dq else 0, self.codes.data_ptr(), q2,
                          self.absmax.data_ptr())
 
     def nbytes(self):
         return self.codes.numel() + self.scale_codes.numel() + 4 * self.absmax.numel()
 
 
-def qlora_quantize_nf4(w, out=None, stream=None):
-    """Quantize a bf16 CUDA weight [N, K] into an :class:`NF4Weight`."""
+def qlora_quantize_nf4(w, out=None, stream=None, dq=True):
+    """Quantize a bf16 CUDA weight [N, K] into an :class:`NF4Weight` (with
+    double quantization unless dq=False or `out` says otherwise)."""
     assert w.is_cuda and w.dim() == 2 and w.is_contiguous()
-    q = out if out is not None else NF4Weight(w.shape[0], w.shape[1], device=w.device)
+    q = out if out is not None else NF4Weight(w.shape[0], w.shape[1], device=w.device, dq=dq)
     s = q.struct()
     _check(lib.qlora_quantize_nf4(_ptr(w), ctypes.byref(s), _stream_ptr(stream)), "qlora_quantize_nf4")
     return q

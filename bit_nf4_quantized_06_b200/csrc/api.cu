@@ -262,9 +262,9 @@ WsPlan plan_ws(int64_t m, int64_t n, int64_t k, int32_t r, int sms, bool fwd_onl
 }
 
 qlora_status_t check_nf4(const qlora_nf4_t* q) {
-  if (q == nullptr || q->codes == nullptr || q->scale_codes == nullptr || q->absmax == nullptr)
-    return QLORA_ERR_INVALID_ARG;
-  if (q->block != kBlock || q->dq_group != kGroup) return QLORA_ERR_INVALID_ARG;
+  if (q == nullptr || q->codes == nullptr || q->absmax == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (q->block != kBlock || (q->dq_group != kGroup && q->dq_group != 0)) return QLORA_ERR_INVALID_ARG;
+  if (q->dq_group == kGroup && q->scale_codes == nullptr) return QLORA_ERR_INVALID_ARG;
   if (q->n_out <= 0 || q->k_in <= 0 || q->k_in % kBlock != 0) return QLORA_ERR_SHAPE;
   if (q->n_out > (int64_t(1) << 31) - 1 || q->k_in > (int64_t(1) << 31) - 1) return QLORA_ERR_SHAPE;
   if (!aligned16(q->codes)) return QLORA_ERR_ALIGNMENT;
@@ -447,11 +447,12 @@ qlora_status_t qlora_nf4_codebook(float out[16]) {
 }
 
 size_t qlora_nf4_bytes(int64_t n_out, int64_t k_in, int32_t dq_group, size_t out[3]) {
-  if (n_out <= 0 || k_in <= 0 || k_in % kBlock != 0 || dq_group != kGroup) return 0;
+  if (n_out <= 0 || k_in <= 0 || k_in % kBlock != 0 || (dq_group != kGroup && dq_group != 0)) return 0;
   const int64_t nb = n_out * k_in / kBlock;
+  const bool dq = dq_group == kGroup;
   const size_t b0 = static_cast<size_t>(n_out * k_in / 2);
-  const size_t b1 = static_cast<size_t>(nb);
-  const size_t b2 = static_cast<size_t>(cdiv(nb, kGroup)) * sizeof(float);
+  const size_t b1 = dq ? static_cast<size_t>(nb) : 0;
+  const size_t b2 = static_cast<size_t>(dq ? cdiv(nb, kGroup) : nb) * sizeof(float);
   if (out) {
     out[0] = b0;
     out[1] = b1;
@@ -492,6 +493,7 @@ qlora_status_t qlora_quantize_nf4(const void* w_bf16, const qlora_nf4_t* q, void
   const int64_t nb = q->n_out * q->k_in / kBlock;
   QuantParams qp{};
   std::memcpy(qp.cut, tables().cut, sizeof(qp.cut));
+  qp.dq = q->dq_group == kGroup ? 1 : 0;
   const int64_t groups = cdiv(nb, kGroup);
   if (groups > 0x7FFFFFFF) return QLORA_ERR_SHAPE;
   k_quantize_nf4<<<static_cast<unsigned>(groups), 256, 0, static_cast<cudaStream_t>(stream)>>>(
@@ -510,6 +512,7 @@ qlora_status_t qlora_dequantize(const qlora_nf4_t* q, void* w_bf16_out, void* st
   const int64_t nwords = q->n_out * q->k_in / 8;
   DequantParams dp{};
   std::memcpy(dp.cb, tables().cb, sizeof(dp.cb));
+  dp.dq = q->dq_group == kGroup ? 1 : 0;
   const int blocks = static_cast<int>(std::min<int64_t>(cdiv(nwords, 256), int64_t(sms) * 16));
   k_dequantize_nf4<<<std::max(blocks, 1), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const uint32_t*>(q->codes), q->scale_codes, q->absmax, nwords,
@@ -601,6 +604,7 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
     gp.r64 = r64;
     gp.ldb = static_cast<int32_t>(ldb);
     std::memcpy(gp.cb, tables().cb, sizeof(gp.cb));
+    gp.dq = q->dq_group == kGroup ? 1 : 0;
     // launched as a programmatic dependent of the x A^T kernel: its weight
     // stream starts while u' is still being computed
     cudaLaunchConfig_t cfg = {};
@@ -645,6 +649,7 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
   p.smax = q->absmax;
   p.kblocks = k / 64;
   p.nblocks = n * (k / 64);
+  p.dq = q->dq_group == kGroup ? 1 : 0;
   p.w_rows = n;
   p.w_cols = k;
   std::memcpy(p.cb, tables().cb, sizeof(p.cb));
@@ -758,6 +763,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
     p.smax = q->absmax;
     p.kblocks = k / 64;
     p.nblocks = n * (k / 64);
+    p.dq = q->dq_group == kGroup ? 1 : 0;
     p.w_rows = n;
     p.w_cols = k;
     std::memcpy(p.cb, tables().cb, sizeof(p.cb));
@@ -813,6 +819,7 @@ qlora_status_t qlora_merge_lora(const qlora_nf4_t* q, const void* a, const void*
   p.r64 = r64_of(r);
   p.s = alpha / static_cast<float>(r);
   std::memcpy(p.cb, tables().cb, sizeof(p.cb));
+  p.dq = q->dq_group == kGroup ? 1 : 0;
   const size_t smem = merge_smem_bytes(p.r64);
   const dim3 grid(static_cast<unsigned>(cdiv(p.k, 128)), static_cast<unsigned>(cdiv(p.n, 128)), 1);
   if (grid.y > 65535u) return QLORA_ERR_SHAPE;

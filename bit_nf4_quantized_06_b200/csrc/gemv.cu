@@ -115,16 +115,24 @@ __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
       ch.a_lo = ldg_stream(src);
       ch.a_hi = ldg_stream(src + 16);
       const int64_t bi = r0 * kpr + kb;
-      ch.q2a = __ldg(p.q2 + bi);
-      ch.sma = __ldg(p.smax + (bi >> 8));
+      if (p.dq) {
+        ch.q2a = __ldg(p.q2 + bi);
+        ch.sma = __ldg(p.smax + (bi >> 8));
+      } else {
+        ch.sma = __ldg(p.smax + bi);     // fp32 block scale, no double quantization
+      }
     }
     if (kv && v1) {
       const uint8_t* src = p.codes + r1 * row_bytes + kb * 32;
       ch.b_lo = ldg_stream(src);
       ch.b_hi = ldg_stream(src + 16);
       const int64_t bi = r1 * kpr + kb;
-      ch.q2b = __ldg(p.q2 + bi);
-      ch.smb = __ldg(p.smax + (bi >> 8));
+      if (p.dq) {
+        ch.q2b = __ldg(p.q2 + bi);
+        ch.smb = __ldg(p.smax + (bi >> 8));
+      } else {
+        ch.smb = __ldg(p.smax + bi);     // fp32 block scale, no double quantization
+      }
     }
   };
 
@@ -138,8 +146,8 @@ __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
   for (int64_t c = warp; c < nchunks; c += WARPS) {
     const int64_t kb = c * 4 + qd;
     const bool kv = kb < kpr;
-    const Nf4Table t0 = make_table(p.cb, restored_scale(cur.q2a, cur.sma));
-    const Nf4Table t1 = make_table(p.cb, restored_scale(cur.q2b, cur.smb));
+    const Nf4Table t0 = make_table(p.cb, p.dq ? restored_scale(cur.q2a, cur.sma) : cur.sma);
+    const Nf4Table t1 = make_table(p.cb, p.dq ? restored_scale(cur.q2b, cur.smb) : cur.smb);
     const uint32_t wa[8] = {cur.a_lo.x, cur.a_lo.y, cur.a_lo.z, cur.a_lo.w,
                             cur.a_hi.x, cur.a_hi.y, cur.a_hi.z, cur.a_hi.w};
     const uint32_t wb[8] = {cur.b_lo.x, cur.b_lo.y, cur.b_lo.z, cur.b_lo.w,

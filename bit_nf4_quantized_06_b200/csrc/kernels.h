@@ -13,6 +13,7 @@ namespace qlora {
 extern __device__ unsigned int g_dev_status;
 
 struct QuantParams {
+  int32_t dq;     // 1: q2 codes + group s_max; 0: fp32 block scale into absmax
   // cut[j] (j < 15): the real number halfway between m_j (the fp32 midpoint
   // of levels j and j+1) and the next float32 above m_j; a quotient rounds
   // to a float32 above m_j exactly when it exceeds cut[j]. cut[15] is padding.
@@ -21,6 +22,7 @@ struct QuantParams {
 
 struct DequantParams {
   float cb[16];   // the 16 fp32 levels
+  int32_t dq;     // 1: s_hat from q2 and s_max; 0: absmax holds s_b per block
 };
 
 __global__ void k_quantize_nf4(const uint4* __restrict__ w, int64_t nb, uint32_t* __restrict__ codes,
@@ -41,6 +43,7 @@ struct GemvParams {
   __nv_bfloat16* y;       // [M x N]
   int64_t n, k;
   int32_t m, r, r64, ldb;
+  int32_t dq;             // 1: s_hat from q2 and s_max; 0: smax holds s_b per block
   float cb[16];
 };
 
@@ -81,6 +84,7 @@ struct TcParams {
   const float* smax;
   int64_t kblocks;      // K/64 of the weight: blocks per weight row
   int64_t nblocks;      // N*K/64: length of q2
+  int32_t dq;           // 1: s_hat from q2 and s_max; 0: smax holds s_b per block
   int64_t w_rows;       // N of the weight (rows of W)
   int64_t w_cols;       // K of the weight
   float cb[16];
@@ -167,6 +171,7 @@ struct MergeParams {
   int64_t n, k;
   int32_t r, r64;
   float s;
+  int32_t dq;               // 1: s_hat from q2 and s_max; 0: smax holds s_b per block
   float cb[16];
 };
 __global__ void k_merge_lora(MergeParams p);

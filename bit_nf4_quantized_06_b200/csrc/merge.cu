@@ -90,8 +90,12 @@ __global__ void __launch_bounds__(256, 2) k_merge_lora(MergeParams p) {
       const int64_t e0 = n * p.k + kc;
       cw[it] = __ldcs(reinterpret_cast<const uint32_t*>(p.codes) + (e0 >> 3));
       const int64_t blk = n * kpr + (kc >> 6);
-      cq2[it] = __ldg(p.q2 + blk);
-      csm[it] = __ldg(p.smax + (blk >> 8));
+      if (p.dq) {
+        cq2[it] = __ldg(p.q2 + blk);
+        csm[it] = __ldg(p.smax + (blk >> 8));
+      } else {
+        csm[it] = __ldg(p.smax + blk);     // fp32 block scale, no double quantization
+      }
     }
   }
 
@@ -206,7 +210,7 @@ __global__ void __launch_bounds__(256, 2) k_merge_lora(MergeParams p) {
     if (n >= p.n || kc >= p.k) continue;
     const int64_t e0 = n * p.k + kc;                 // first element of the chunk
     const uint32_t w = cw[it];
-    const float sh = restored_scale(cq2[it], csm[it]);
+    const float sh = p.dq ? restored_scale(cq2[it], csm[it]) : csm[it];
     const float4 dlo = *reinterpret_cast<const float4*>(sD + row * LDD + c8 * 8);
     const float4 dhi = *reinterpret_cast<const float4*>(sD + row * LDD + c8 * 8 + 4);
     const float d[8] = {dlo.x, dlo.y, dlo.z, dlo.w, dhi.x, dhi.y, dhi.z, dhi.w};

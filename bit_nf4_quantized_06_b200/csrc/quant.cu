@@ -106,9 +106,20 @@ __global__ void __launch_bounds__(256) k_quantize_nf4(const uint4* __restrict__ 
 #pragma unroll
   for (int i = 1; i < 8; ++i) gmax = max(gmax, s_wmax[i]);
   const float s_max = __uint_as_float(gmax << 16);
-  if (tid == 0) smax[g] = s_max;
+  if (!qp.dq) {
+    // 4.5-bit format: the block scale itself is stored (exact: a bf16 magnitude)
+    if ((tid & 7) == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int bi = (tid >> 3) + 32 * i;
+        if (bi < nblk) smax[b0 + bi] = __uint_as_float(am[i] << 16);
+      }
+    }
+  } else if (tid == 0) {
+    smax[g] = s_max;
+  }
 
-  if ((tid & 7) == 0) {
+  if (qp.dq && (tid & 7) == 0) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int bi = (tid >> 3) + 32 * i;
@@ -166,7 +177,7 @@ __global__ void __launch_bounds__(256) k_dequantize_nf4(const uint32_t* __restri
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nwords;
        i += stride) {
     const int64_t b = i >> 3;
-    const float s_hat = restored_scale(__ldg(q2 + b), __ldg(smax + (b >> 8)));
+    const float s_hat = dp.dq ? restored_scale(__ldg(q2 + b), __ldg(smax + (b >> 8))) : __ldg(smax + b);
     const uint32_t w = __ldcs(codes + i);
     uint32_t o[4];
 #pragma unroll

@@ -246,13 +246,16 @@ __global__ void __launch_bounds__(448, 1)
       if (c.j < items && c.t < p.kt_main) {
         const int64_t bi = block_of(c.f0, c.t);
         const uint32_t slot = slot0 + k * (128 * 8);
-        if (bi >= 0) {
+        if (bi >= 0 && p.dq) {
           const int64_t w4 = bi & ~int64_t(3);
           const int64_t left = p.nblocks - w4;
           cp_async4(slot, p.q2 + w4, static_cast<uint32_t>(left < 4 ? left : 4));
           cp_async4(slot + 4, p.smax + (bi >> 8), 4);
+        } else if (bi >= 0) {
+          cp_async4(slot, p.smax, 0);
+          cp_async4(slot + 4, p.smax + bi, 4);     // fp32 block scale, no double quantization
         } else {
-          cp_async4(slot, p.q2, 0);
+          cp_async4(slot, p.smax, 0);
           cp_async4(slot + 4, p.smax, 0);
         }
       }
@@ -295,9 +298,13 @@ __global__ void __launch_bounds__(448, 1)
         const uint32_t slot = slot0 + slot_use * (128 * 8);
         float sh = 0.0f;
         if (bi >= 0) {
-          const uint32_t qw = lds32(slot);
-          const uint32_t q2 = (qw >> (8 * static_cast<uint32_t>(bi & 3))) & 0xFFu;
-          sh = restored_scale(q2, __uint_as_float(lds32(slot + 4)));
+          if (p.dq) {
+            const uint32_t qw = lds32(slot);
+            const uint32_t q2 = (qw >> (8 * static_cast<uint32_t>(bi & 3))) & 0xFFu;
+            sh = restored_scale(q2, __uint_as_float(lds32(slot + 4)));
+          } else {
+            sh = __uint_as_float(lds32(slot + 4));
+          }
         }
         const Nf4Table tb = make_table(p.cb, sh);
         ok = mbar_wait(bar_codes(s), ph, abort_flag, QLORA_DEV_TIMEOUT_APROD);

@@ -78,23 +78,32 @@ typedef enum {
   QLORA_ERR_TIMEOUT = 7            /* a kernel gave up on a bounded wait            */
 } qlora_status_t;
 
-/* Packed NF4 weight with double-quantized scales. All pointers are device
- * pointers owned by the caller; sizes from qlora_nf4_bytes(). */
+/* Packed NF4 weight. All pointers are device pointers owned by the caller;
+ * sizes from qlora_nf4_bytes(). Two formats («QLoRA는 어떻게 65B 모델을 GPU 한
+ * 장에 올렸나», § "메모리 회계: 세 겹의 최적화"):
+ *   dq_group = 256: double quantization (~4.13 bits/param): scale_codes holds
+ *     one 8-bit code q2 per 64-weight block and absmax one fp32 s_max per 256
+ *     consecutive blocks; the block scale is s_hat = fl32(q2 * s_max) * 2^-8;
+ *   dq_group = 0: no double quantization (4.5 bits/param): absmax holds the
+ *     fp32 block scale s_b itself, one per block; scale_codes is unused and
+ *     may be NULL. */
 typedef struct {
   int64_t n_out;         /* N rows (d_out)                                     */
   int64_t k_in;          /* K columns (d_in), K % 64 == 0                      */
   int32_t block;         /* weights per absmax block: must be 64               */
-  int32_t dq_group;      /* blocks per double-quantization group: must be 256 */
+  int32_t dq_group;      /* 256 (double quantization) or 0 (none)              */
   uint8_t *codes;        /* N*K/2 bytes                                        */
-  uint8_t *scale_codes;  /* N*K/64 bytes                                       */
-  float *absmax;         /* ceil(N*K/64/256) floats: the group constants s_max */
+  uint8_t *scale_codes;  /* N*K/64 bytes (dq_group 256), unused for 0          */
+  float *absmax;         /* ceil(N*K/64/256) s_max (dq_group 256), or N*K/64
+                            block scales (dq_group 0)                          */
 } qlora_nf4_t;
 
 /* Forward path selection for qlora_linear_fwd_ex. AUTO takes the decode GEMV
  * for m <= 16 and the tensor-core GEMM otherwise. */
 typedef enum { QLORA_FWD_AUTO = 0, QLORA_FWD_GEMM = 1, QLORA_FWD_GEMV = 2 } qlora_fwd_path_t;
 
-/* Byte sizes of the three stored arrays; returns their sum (0 on bad shape).
+/* Byte sizes of the three stored arrays (codes, scale codes, fp32 scales)
+ * for dq_group 256 or 0; returns their sum (0 on bad shape or dq_group).
  * out may be NULL. Host only, no device work. */
 QLORA_API size_t qlora_nf4_bytes(int64_t n_out, int64_t k_in, int32_t dq_group, size_t out[3]);
 

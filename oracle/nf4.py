@@ -183,6 +183,21 @@ def dequantize(codes, q2, smax):
     return bf16_bits_to_f32(dequantize_bits(codes, q2, smax))
 
 
+def dequantize_bits_no_dq(codes, absmax):
+    """Restore without double quantization (the 4.5-bit format: one fp32
+    scale per block, «QLoRA는 어떻게 65B 모델을 GPU 한 장에 올렸나», § "메모리 회계"):
+    w_hat = bf16_rne(fl32(c[q] * s_b)), uint16 [N, K]."""
+    q = unpack(codes)
+    n, k = q.shape
+    c = codebook()
+    prod = (c[q].reshape(-1, BLOCK) * np.asarray(absmax, dtype=np.float32).reshape(-1, 1)).astype(np.float32)
+    return round_f32_to_bf16_bits(prod).reshape(n, k)
+
+
+def dequantize_no_dq(codes, absmax):
+    return bf16_bits_to_f32(dequantize_bits_no_dq(codes, absmax))
+
+
 def storage_bytes(n, k, dq=True):
     """Bytes of the stored format: (codes, scale codes or fp32 scales, group constants)."""
     nb = n * k // BLOCK

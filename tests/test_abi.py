@@ -110,3 +110,13 @@ def test_adamw_argument_validation(q):
     assert lib.qlora_adamw_step(f, None, f, f, f, 0, ctypes.byref(hp), None) == 0   # nothing to do
     hp.beta1 = 1.0
     assert lib.qlora_adamw_step(f, None, f, f, f, 10, ctypes.byref(hp), None) == 1
+
+
+def test_nf4_bytes_without_double_quantization(q):
+    c, q2, sc = q.qlora_nf4_bytes(4096, 4096, 0)
+    assert (c, q2, sc) == (4096 * 4096 // 2, 0, 4 * 4096 * 4096 // 64)
+    assert 8 * (c + q2 + sc) / (4096 * 4096) == 4.5
+    s = q.Nf4Struct(512, 512, 64, 128, 16, 16, 16)          # dq_group must be 256 or 0
+    assert q.lib.qlora_dequantize(ctypes.byref(s), ctypes.c_void_p(16), None) == 1
+    s = q.Nf4Struct(512, 512, 64, 0, 16, 0, 16)             # no scale codes needed without DQ
+    assert q.lib.qlora_dequantize(ctypes.byref(s), None, None) == 1   # (null output still rejected)

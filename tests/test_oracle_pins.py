@@ -406,3 +406,21 @@ def test_adamw_matches_torch_adamw():
         tp.grad = torch.tensor(g, dtype=torch.float64)
         opt.step()
     assert np.allclose(p, tp.detach().numpy(), rtol=1e-13, atol=1e-15)
+
+
+# --------------------------------------------------------------------------- format without double quantization
+
+def test_no_dq_restore_matches_brute_force_and_bound():
+    # 4.5-bit format: the block scale is stored as fp32 and used as is
+    w = synth.weight(6, 128, seed=31, outliers=True).float().numpy()
+    o = nf4.quantize(w)
+    got = nf4.dequantize_no_dq(o["codes"], o["absmax"])
+    levels = [float(x) for x in nf4.codebook()]
+    for i in range(6):
+        for j in range(128):
+            b = (i * 128 + j) // 64
+            expect = bf16.round_to_bf16(np.float32(levels[o["q"][i, j]]) * np.float32(o["absmax"][b]))
+            assert got[i, j] == expect
+    # error within half the largest level gap of the block scale, plus bf16 rounding
+    s_b = np.repeat(o["absmax"].reshape(6, 2), 64, axis=1)
+    assert np.all(np.abs(w - got) <= s_b * nf4.max_level_gap() / 2 + np.abs(got) * 2.0 ** -8 + 1e-30)
