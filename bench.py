@@ -411,6 +411,57 @@ def paged_optimizer(q, wl, l2, reps=10):
                       "of the backward; medians of 10"}
 
 
+def fused_siblings(q, device, l2, reps=5):
+    """7B attention q, k, v (3 x 4096x4096, r = 64 each, 4096 tokens):
+    forward + backward as three separate calls vs one call on the weights
+    concatenated along d_out, adapters stacked along the rank and B block
+    diagonal (x and x A^T streamed once)."""
+    k, n, r, m, alpha = 4096, 4096, 64, 4096, 16.0
+    ws = [synth.weight(n, k, seed=40 + i).to(device) for i in range(3)]
+    As = [synth.lora_a(r, k, seed=50 + i).to(device) for i in range(3)]
+    Bs = [synth.lora_b(n, r, seed=60 + i).to(device) for i in range(3)]
+    x = synth.tokens(m, k, seed=7).to(device)
+    dy = synth.grad_out(m, 3 * n, seed=8).to(device)
+    qws = [q.qlora_quantize_nf4(w) for w in ws]
+    qc = q.qlora_quantize_nf4(torch.cat(ws, 0))
+    a_cat = torch.cat(As, 0)
+    b_bd = torch.zeros((3 * n, 3 * r), dtype=torch.bfloat16, device=device)
+    for i in range(3):
+        b_bd[i * n:(i + 1) * n, i * r:(i + 1) * r] = Bs[i]
+    dys = [dy[:, i * n:(i + 1) * n].contiguous() for i in range(3)]
+    ws1 = torch.empty(q.qlora_workspace_bytes(m, n, k, r) + 256, dtype=torch.uint8, device=device)
+    ws3 = torch.empty(q.qlora_workspace_bytes(m, 3 * n, k, 3 * r) + 256, dtype=torch.uint8, device=device)
+
+    def separate():
+        for i in range(3):
+            y, u = q.qlora_linear_fwd(qws[i], x, As[i], Bs[i], alpha, ws=ws1)
+            q.qlora_linear_bwd(qws[i], x, u, dys[i], As[i], Bs[i], alpha, ws=ws1)
+
+    def fused():
+        y, u = q.qlora_linear_fwd(qc, x, a_cat, b_bd, 3 * alpha, ws=ws3)
+        q.qlora_linear_bwd(qc, x, u, dy, a_cat, b_bd, 3 * alpha, ws=ws3)
+
+    out = {}
+    for name, fn in (("separate", separate), ("fused", fused)):
+        fn()
+        ts = []
+        for _ in range(reps):
+            flush_l2(l2)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        out[name + "_ms"] = round(float(np.median(ts)), 4)
+    fl = 3 * (fwd_flops(m, n, k, r) + bwd_flops(m, n, k, r))
+    out["separate_TFLOP/s"] = round(fl / (out["separate_ms"] * 1e-3) / 1e12, 1)
+    out["fused_TFLOP/s"] = round(fl / (out["fused_ms"] * 1e-3) / 1e12, 1)
+    out["speedup"] = round(out["separate_ms"] / out["fused_ms"], 3)
+    out["workload"] = "7B attention q,k,v: 3 x 4096x4096 NF4, r=64 each, 4096 tokens, fwd+bwd"
+    return out
+
+
 def cpu_baseline_sample(target_s=15.0):
     """Time the oracle (as it stands) on a bounded sample of the same step:
     quantize the full W, forward + backward for `tok` tokens (fp64)."""
@@ -507,6 +558,7 @@ def run_ours(args):
     # LoRA merge for export and the paged adapter optimizer (outside the step)
     merge_ms, mb = merge_timing(q, wl, l2)
     popt = paged_optimizer(q, wl, l2)
+    sib = fused_siblings(q, device, l2)
 
     # decode GEMV steady state + single-call latency
     gemv_ms, gemv_lat_ms, _ = gemv_steady_state(q, device)
@@ -576,6 +628,7 @@ def run_ours(args):
                   "frac_hbm": round(mb / (merge_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                   "method": "median of 10 calls, L2 flushed before each"},
         "paged_optimizer": popt,
+        "fused_siblings": sib,
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
