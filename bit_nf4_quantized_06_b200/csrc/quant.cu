@@ -42,25 +42,43 @@ __device__ __forceinline__ uint32_t abs_bits_max(uint4 v) {
   return m;
 }
 
+// Exact code of one weight by the division-free test: for a bf16 weight w
+// and a block scale s > 0,
+//   fl32(w / s) > m_j   <=>   w / s > m'_j   <=>   w > m'_j * s   <=>   w > RD_bf16(m'_j * s)
+// where m'_j (cut[j]) is the midpoint between m_j and the next float32 above
+// it. Round-to-nearest sends w / s above m_j exactly when w / s exceeds that
+// midpoint; equality would need m'_j * s (a 25-bit odd significand times an
+// 8-bit one) to have at most 8 significant bits, which it cannot; m'_j * s is
+// exact in float64; and because w lies on the bf16 grid, comparing with the
+// product rounded down to that grid gives the same answer.
+__device__ __noinline__ uint32_t exact_code(float w, float s, const double* cut) {
+  uint32_t q = 0;
+  for (int j = 0; j < 15; ++j) {
+    const float t = __bfloat162float(__float2bfloat16_rd(__double2float_rd(cut[j] * static_cast<double>(s))));
+    q += (w > t) ? 1u : 0u;
+  }
+  return q;
+}
+
 }  // namespace
 
 // One CTA of 256 threads per double-quantization group (see the file comment).
 //
-// Encode without dividing: for a bf16 weight w and a block scale s > 0,
-//   fl32(w / s) > m_j   <=>   w / s > m'_j   <=>   w > m'_j * s   <=>   w > RD_bf16(m'_j * s)
-// where m'_j is the midpoint between m_j and the next float32 above it.
-// Round-to-nearest sends w / s above m_j exactly when w / s exceeds that
-// midpoint; equality would need m'_j * s (a 25-bit odd significand times an
-// 8-bit one) to have at most 8 significant bits, which it cannot; m'_j * s is
-// exact in float64; and because w lies on the bf16 grid, comparing with the
-// product rounded down to that grid gives the same answer. So each block
-// computes its 15 thresholds once (two per lane of the 8 lanes that share the
-// block) and every weight is placed by a 4-step binary search over them.
-__global__ void __launch_bounds__(256) k_quantize_nf4(const uint4* __restrict__ w,
+// Encode by cells: with r = fl32(1 / s), the quotient x' = fl32(w * r) lies
+// within 3.0001 * 2^-24 of fl32(w / s) for |w| <= s. Its cell
+// c = rint(128 x' + 128) (0..256, one fused multiply-add around a large
+// constant) selects a table entry holding the number of level midpoints
+// below the cell and the one midpoint m inside it (the cells are narrower
+// than the gaps between midpoints), so q = below + [x' > m] -- exactly the
+// count #{j : fl32(w / s) > m_j} whenever |x' - m| exceeds the guard. The
+// rare weights within the guard of a midpoint, and blocks whose scale is
+// subnormal (1/s may overflow), take the exact test above.
+__global__ void __launch_bounds__(256, 2) k_quantize_nf4(const uint4* __restrict__ w,
                                                       int64_t nb, uint32_t* __restrict__ codes,
                                                       uint8_t* __restrict__ q2,
                                                       float* __restrict__ smax, QuantParams qp) {
-  __shared__ float s_thr[256][17];   // per block: 15 thresholds (+ pad), row stride 17 against bank conflicts
+  __shared__ float2 s_cell[257];
+  __shared__ double s_cut[16];
   __shared__ uint32_t s_wmax[8];
   const int tid = threadIdx.x;
   const int64_t g = blockIdx.x;
@@ -74,6 +92,8 @@ __global__ void __launch_bounds__(256) k_quantize_nf4(const uint4* __restrict__ 
     const int bi = (tid >> 3) + 32 * i;
     v[i] = (bi < nblk) ? __ldcs(w + chunk0 + tid + 256 * i) : make_uint4(0, 0, 0, 0);
   }
+  for (int c = tid; c < 257; c += 256) s_cell[c] = qp.cell[c];
+  if (tid < 16) s_cut[tid] = qp.cut[tid];
 
   uint32_t am[8];
   uint32_t gm = 0;
@@ -89,18 +109,6 @@ __global__ void __launch_bounds__(256) k_quantize_nf4(const uint4* __restrict__ 
   gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 8));
   gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 16));
   if ((tid & 31) == 0) s_wmax[tid >> 5] = gm;
-
-  // thresholds of this lane's share: j = 2 * (tid % 8) and j + 1, for each of its 8 blocks
-  const int j0 = 2 * (tid & 7);
-  const double mp0 = qp.cut[j0];
-  const double mp1 = qp.cut[j0 + 1];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int bi = (tid >> 3) + 32 * i;
-    const double sd = static_cast<double>(__uint_as_float(am[i] << 16));
-    s_thr[bi][j0] = __bfloat162float(__float2bfloat16_rd(__double2float_rd(mp0 * sd)));
-    s_thr[bi][j0 + 1] = __bfloat162float(__float2bfloat16_rd(__double2float_rd(mp1 * sd)));
-  }
   __syncthreads();
   uint32_t gmax = s_wmax[0];
 #pragma unroll
@@ -135,29 +143,51 @@ __global__ void __launch_bounds__(256) k_quantize_nf4(const uint4* __restrict__ 
     }
   }
 
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: the integer part lands in the low mantissa bits
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int bi = (tid >> 3) + 32 * i;
     if (bi < nblk) {
-      const float* t = s_thr[bi];
-      const bool zero = (am[i] == 0);
+      const uint32_t a = am[i];
+      const float sb = __uint_as_float(a << 16);
+      const bool zero = (a == 0);
+      const bool tiny = (a < 0x0080u);     // zero or subnormal scale
+      const float r = tiny ? 0.0f : __frcp_rn(sb);
       const uint32_t ww[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      uint32_t qv[8];
+      bool any_amb = false;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        // element e of the chunk: bf16 pair e/2 holds element 2k in its low half
+        const float we = (e & 1) ? __uint_as_float(ww[e >> 1] & 0xFFFF0000u) : __uint_as_float(ww[e >> 1] << 16);
+        const float x = __fmul_rn(we, r);
+        const float t = fmaf(x, 128.0f, 128.0f + kMagic);
+        const uint32_t c = min(__float_as_uint(t) - __float_as_uint(kMagic), 256u);
+        const float2 cell = s_cell[c];
+        const float d = __fsub_rn(x, cell.x);
+        qv[e] = (__float_as_uint(cell.y) & 0xFFu) + (d > 0.0f ? 1u : 0u);
+        any_amb |= !(fabsf(d) > kEncodeGuard);
+      }
+      if (tiny || any_amb) {
+        // rare: redo the weights near a midpoint (or the whole block) exactly
+#pragma unroll 1
+        for (int e = 0; e < 8; ++e) {
+          const float we = (e & 1) ? __uint_as_float(ww[e >> 1] & 0xFFFF0000u) : __uint_as_float(ww[e >> 1] << 16);
+          if (zero) {
+            qv[e] = 7u;
+          } else if (tiny) {
+            qv[e] = exact_code(we, sb, s_cut);
+          } else {
+            const float x = __fmul_rn(we, r);
+            const float t = fmaf(x, 128.0f, 128.0f + kMagic);
+            const uint32_t c = min(__float_as_uint(t) - __float_as_uint(kMagic), 256u);
+            if (!(fabsf(__fsub_rn(x, s_cell[c].x)) > kEncodeGuard)) qv[e] = exact_code(we, sb, s_cut);
+          }
+        }
+      }
       uint32_t word = 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        // bf16 pair j holds elements 2j (low half) and 2j+1 (high half)
-        const float e[2] = {__uint_as_float(ww[j] << 16), __uint_as_float(ww[j] & 0xFFFF0000u)};
-        uint32_t qq[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t q = (e[h] > t[7]) ? 8u : 0u;
-          q += (e[h] > t[q + 3]) ? 4u : 0u;
-          q += (e[h] > t[q + 1]) ? 2u : 0u;
-          q += (e[h] > t[q]) ? 1u : 0u;
-          qq[h] = zero ? 7u : q;
-        }
-        word |= ((qq[0] << 4) | qq[1]) << (8 * j);
-      }
+      for (int j = 0; j < 4; ++j) word |= ((qv[2 * j] << 4) | qv[2 * j + 1]) << (8 * j);
       codes[chunk0 + tid + 256 * i] = word;
     }
   }

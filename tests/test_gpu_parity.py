@@ -87,6 +87,49 @@ def test_dequantize_bit_exact(q, n, k, outl, seed):
     assert np.array_equal(_bits(wh), nf4.dequantize_bits(o["codes"], o["q2"], o["smax"]))
 
 
+def _near_midpoint_blocks(nblocks, seed):
+    """Blocks whose weights sit on the bf16 grid right at (and one step either
+    side of) m_j * s for every level midpoint m_j, for scales spread over the
+    exponent range, including subnormal ones: every encode decision here is
+    a near tie."""
+    rng = np.random.default_rng(seed)
+    mids = nf4.midpoints().astype(np.float64)
+    rows = []
+    for b in range(nblocks):
+        e = rng.integers(-140, 10) if b % 4 else rng.integers(-133, -126)   # every 4th block: subnormal scale
+        s_val = float(np.ldexp(1.0 + rng.random(), int(e)))
+        s_bits = obf16.round_f32_to_bf16_bits(np.array([s_val], dtype=np.float32))
+        s = float(obf16.bf16_bits_to_f32(s_bits)[0])
+        if s == 0.0:
+            s = float(obf16.bf16_bits_to_f32(np.array([1], dtype=np.uint16))[0])
+        vals = []
+        for m in mids[rng.permutation(15)[:10]]:
+            target = np.float32(m * s)
+            bits = int(obf16.round_f32_to_bf16_bits(np.array([target], dtype=np.float32))[0])
+            for dbits in (-1, 0, 1):
+                vals.append(float(obf16.bf16_bits_to_f32(np.array([(bits + dbits) & 0xFFFF], dtype=np.uint16))[0]))
+        vals = [v for v in vals if abs(v) <= s][:62]
+        while len(vals) < 62:
+            vals.append(float(rng.uniform(-s, s)))
+        blk = np.array([s, -s * 0.5] + vals, dtype=np.float32)[:64]
+        rows.append(rng.permutation(blk))
+    return obf16.round_to_bf16(np.concatenate(rows).astype(np.float32))
+
+
+def test_quantize_near_midpoints_bit_exact(q):
+    n, k = 64, 1024                                   # 1024 blocks, 4 groups
+    w = _near_midpoint_blocks(n * k // 64, seed=3).reshape(n, k)
+    o = nf4.quantize(w)
+    qw = q.qlora_quantize_nf4(torch.from_numpy(w).to(torch.bfloat16).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(qw.codes.cpu().numpy(), o["codes"].ravel())
+    assert np.array_equal(qw.scale_codes.cpu().numpy(), o["q2"])
+    qn = q.qlora_quantize_nf4(torch.from_numpy(w).to(torch.bfloat16).cuda(), dq=False)
+    torch.cuda.synchronize()
+    assert np.array_equal(qn.codes.cpu().numpy(), o["codes"].ravel())
+    assert np.array_equal(qn.absmax.cpu().numpy().view(np.uint32), o["absmax"].view(np.uint32))
+
+
 def test_quantize_full_size_7b_mlp(q):
     p = synth.MLP7B
     w = synth.weight(p.n, p.k)
