@@ -44,7 +44,8 @@ struct Tables {
   float cb[16];
   float mid[16];
   double cut[16];
-  float2 cell[257];
+  float cell_m[33];
+  uint32_t cell_info[33];
 };
 
 const Tables& tables() {
@@ -69,20 +70,19 @@ const Tables& tables() {
     for (int i = 0; i < 15; ++i)
       r.cut[i] = (static_cast<double>(r.mid[i]) + static_cast<double>(std::nextafter(r.mid[i], 2.0f))) / 2.0;
     r.cut[15] = 2.0;
-    // encoder cells: cell c covers x in [(c - 128.5) / 128, (c - 127.5) / 128],
+    // encoder cells: cell c covers x in [(c - 16.5) / 16, (c - 15.5) / 16],
     // widened by twice the guard; at most one midpoint falls in a widened cell
-    // (the midpoints are more than 0.07 apart, a cell is 0.0078 wide)
+    // (the midpoints are more than 0.08 apart, a cell is 0.0625 wide)
     const double g2 = 2.0 * static_cast<double>(kEncodeGuard);
-    for (int c = 0; c <= 256; ++c) {
-      const double lo = (c - 128.5) / 128.0 - g2, hi = (c - 127.5) / 128.0 + g2;
+    for (int c = 0; c <= 32; ++c) {
+      const double lo = (c - 16.5) / 16.0 - g2, hi = (c - 15.5) / 16.0 + g2;
       int below = 0, cand = -1;
       for (int j = 0; j < 15; ++j) {
         if (r.mid[j] < lo) ++below;
         else if (r.mid[j] <= hi) cand = j;
       }
-      r.cell[c].x = cand >= 0 ? r.mid[cand] : 4.0f;
-      uint32_t packed = static_cast<uint32_t>(below) | (static_cast<uint32_t>(cand >= 0 ? cand : 15) << 8);
-      std::memcpy(&r.cell[c].y, &packed, 4);
+      r.cell_m[c] = cand >= 0 ? r.mid[cand] : 4.0f;
+      r.cell_info[c] = static_cast<uint32_t>(below) | (static_cast<uint32_t>(cand >= 0 ? cand : 15) << 8);
     }
     return r;
   }();
@@ -509,7 +509,8 @@ qlora_status_t qlora_quantize_nf4(const void* w_bf16, const qlora_nf4_t* q, void
   const int64_t nb = q->n_out * q->k_in / kBlock;
   QuantParams qp{};
   std::memcpy(qp.cut, tables().cut, sizeof(qp.cut));
-  std::memcpy(qp.cell, tables().cell, sizeof(qp.cell));
+  std::memcpy(qp.cell_m, tables().cell_m, sizeof(qp.cell_m));
+  std::memcpy(qp.cell_info, tables().cell_info, sizeof(qp.cell_info));
   qp.dq = q->dq_group == kGroup ? 1 : 0;
   const int64_t groups = cdiv(nb, kGroup);
   if (groups > 0x7FFFFFFF) return QLORA_ERR_SHAPE;

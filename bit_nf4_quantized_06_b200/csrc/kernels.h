@@ -18,11 +18,13 @@ struct QuantParams {
   // of levels j and j+1) and the next float32 above m_j; a quotient rounds
   // to a float32 above m_j exactly when it exceeds cut[j]. cut[15] is padding.
   double cut[16];
-  // Cell table of the encoder: cell c (0..256) holds the quotients x with
-  // rint(128 x + 128) == c, widened by the guard below; cell[c].x is the one
-  // level midpoint m_j inside the widened cell (or 4.0 if there is none) and
-  // cell[c].y packs (number of midpoints below the widened cell) | (j << 8).
-  float2 cell[257];
+  // Cell table of the encoder: cell c (0..32) holds the quotients x with
+  // rint(16 x + 16) == c, widened by twice the guard below; cell_m[c] is the
+  // one level midpoint m_j inside the widened cell (4.0 if there is none) and
+  // cell_info[c] packs (number of midpoints below the widened cell) | (j << 8).
+  // A cell is 1/16 wide and the midpoints are more than 0.08 apart.
+  float cell_m[33];
+  uint32_t cell_info[33];
 };
 // |fl32(w * fl32(1/s)) - fl32(w / s)| <= 3.0001 * 2^-24 for |w| <= s; a
 // quotient farther than this guard from the candidate midpoint is decided

@@ -66,18 +66,21 @@ __device__ __noinline__ uint32_t exact_code(float w, float s, const double* cut)
 //
 // Encode by cells: with r = fl32(1 / s), the quotient x' = fl32(w * r) lies
 // within 3.0001 * 2^-24 of fl32(w / s) for |w| <= s. Its cell
-// c = rint(128 x' + 128) (0..256, one fused multiply-add around a large
+// c = rint(16 x' + 16) (0..32, one fused multiply-add around a large
 // constant) selects a table entry holding the number of level midpoints
-// below the cell and the one midpoint m inside it (the cells are narrower
-// than the gaps between midpoints), so q = below + [x' > m] -- exactly the
-// count #{j : fl32(w / s) > m_j} whenever |x' - m| exceeds the guard. The
-// rare weights within the guard of a midpoint, and blocks whose scale is
-// subnormal (1/s may overflow), take the exact test above.
-__global__ void __launch_bounds__(256, 2) k_quantize_nf4(const uint4* __restrict__ w,
+// below the cell and the one midpoint m inside it (a cell is narrower than
+// the gaps between midpoints), so q = below + [x' > m] -- exactly the count
+// #{j : fl32(w / s) > m_j} whenever |x' - m| exceeds the guard. The two
+// 33-word tables sit in shared memory, one word per bank, so the lookups
+// never conflict. The rare weights within the guard of a midpoint, and
+// blocks whose scale is subnormal (1/s may overflow), take the exact test
+// above.
+__global__ void __launch_bounds__(256, 3) k_quantize_nf4(const uint4* __restrict__ w,
                                                       int64_t nb, uint32_t* __restrict__ codes,
                                                       uint8_t* __restrict__ q2,
                                                       float* __restrict__ smax, QuantParams qp) {
-  __shared__ float2 s_cell[257];
+  __shared__ float s_cm[33];
+  __shared__ uint32_t s_ci[33];
   __shared__ double s_cut[16];
   __shared__ uint32_t s_wmax[8];
   const int tid = threadIdx.x;
@@ -92,7 +95,10 @@ __global__ void __launch_bounds__(256, 2) k_quantize_nf4(const uint4* __restrict
     const int bi = (tid >> 3) + 32 * i;
     v[i] = (bi < nblk) ? __ldcs(w + chunk0 + tid + 256 * i) : make_uint4(0, 0, 0, 0);
   }
-  for (int c = tid; c < 257; c += 256) s_cell[c] = qp.cell[c];
+  if (tid < 33) {
+    s_cm[tid] = qp.cell_m[tid];
+    s_ci[tid] = qp.cell_info[tid];
+  }
   if (tid < 16) s_cut[tid] = qp.cut[tid];
 
   uint32_t am[8];
@@ -161,11 +167,10 @@ __global__ void __launch_bounds__(256, 2) k_quantize_nf4(const uint4* __restrict
         // element e of the chunk: bf16 pair e/2 holds element 2k in its low half
         const float we = (e & 1) ? __uint_as_float(ww[e >> 1] & 0xFFFF0000u) : __uint_as_float(ww[e >> 1] << 16);
         const float x = __fmul_rn(we, r);
-        const float t = fmaf(x, 128.0f, 128.0f + kMagic);
-        const uint32_t c = min(__float_as_uint(t) - __float_as_uint(kMagic), 256u);
-        const float2 cell = s_cell[c];
-        const float d = __fsub_rn(x, cell.x);
-        qv[e] = (__float_as_uint(cell.y) & 0xFFu) + (d > 0.0f ? 1u : 0u);
+        const float t = fmaf(x, 16.0f, 16.0f + kMagic);
+        const uint32_t c = min(__float_as_uint(t) - __float_as_uint(kMagic), 32u);
+        const float d = __fsub_rn(x, s_cm[c]);
+        qv[e] = (s_ci[c] & 0xFFu) + (d > 0.0f ? 1u : 0u);
         any_amb |= !(fabsf(d) > kEncodeGuard);
       }
       if (tiny || any_amb) {
@@ -179,9 +184,9 @@ __global__ void __launch_bounds__(256, 2) k_quantize_nf4(const uint4* __restrict
             qv[e] = exact_code(we, sb, s_cut);
           } else {
             const float x = __fmul_rn(we, r);
-            const float t = fmaf(x, 128.0f, 128.0f + kMagic);
-            const uint32_t c = min(__float_as_uint(t) - __float_as_uint(kMagic), 256u);
-            if (!(fabsf(__fsub_rn(x, s_cell[c].x)) > kEncodeGuard)) qv[e] = exact_code(we, sb, s_cut);
+            const float t = fmaf(x, 16.0f, 16.0f + kMagic);
+            const uint32_t c = min(__float_as_uint(t) - __float_as_uint(kMagic), 32u);
+            if (!(fabsf(__fsub_rn(x, s_cm[c])) > kEncodeGuard)) qv[e] = exact_code(we, sb, s_cut);
           }
         }
       }
