@@ -462,6 +462,69 @@ def fused_siblings(q, device, l2, reps=5):
     return out
 
 
+def whole_stack(q, device, l2):
+    """The whole 7B-shaped stack: 32 layers of q, k, v, o (4096x4096), gate,
+    up (11008x4096) and down (4096x11008), 6,476,005,376 weights ~ N(0, 0.02).
+    Each weight is generated on the GPU from its own seed, quantized (NF4 +
+    double quantization; CUDA events around the quantize calls only) and its
+    bf16 copy freed. Then forward + backward of all 224 quantized linears at
+    4096 tokens with r = 64 adapters, one event pair around the whole sweep."""
+    m, r, alpha = 4096, 64, 16.0
+    gen = torch.Generator(device=device)
+    lin, params, q_ms = [], 0, 0.0
+    for layer in range(synth.STACK7B_LAYERS):
+        for idx, (_, n, k) in enumerate(synth.STACK7B_LAYER):
+            gen.manual_seed(10_000 + 16 * layer + idx)
+            w = (torch.randn((n, k), generator=gen, device=device) * 0.02).to(torch.bfloat16)
+            qw = q.NF4Weight(n, k, device=device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            q.qlora_quantize_nf4(w, out=qw)
+            e1.record()
+            torch.cuda.synchronize()
+            q_ms += e0.elapsed_time(e1)
+            del w
+            a = (torch.rand((r, k), generator=gen, device=device) * 2 - 1).mul_(k ** -0.5).to(torch.bfloat16)
+            b = (torch.randn((n, r), generator=gen, device=device) * 0.01).to(torch.bfloat16)
+            lin.append((qw, n, k, a, b))
+            params += n * k
+    xs = {k: torch.randn((m, k), generator=gen, device=device).to(torch.bfloat16) for k in (4096, 11008)}
+    dys = {n: torch.randn((m, n), generator=gen, device=device).to(torch.bfloat16) for n in (4096, 11008)}
+    ys = {n: torch.empty((m, n), dtype=torch.bfloat16, device=device) for n in (4096, 11008)}
+    dxs = {k: torch.empty((m, k), dtype=torch.bfloat16, device=device) for k in (4096, 11008)}
+    u = torch.empty((m, r), dtype=torch.bfloat16, device=device)
+    das = {k: torch.empty((r, k), dtype=torch.float32, device=device) for k in (4096, 11008)}
+    dbs = {n: torch.empty((n, r), dtype=torch.float32, device=device) for n in (4096, 11008)}
+    ws = torch.empty(max(q.qlora_workspace_bytes(m, n, k, r) for _, n, k, _, _ in lin) + 256, dtype=torch.uint8,
+                     device=device)
+
+    def sweep():
+        for qw, n, k, a, b in lin:
+            q.qlora_linear_fwd(qw, xs[k], a, b, alpha, y=ys[n], u=u, ws=ws)
+            q.qlora_linear_bwd(qw, xs[k], u, dys[n], a, b, alpha, dx=dxs[k], da=das[k], db=dbs[n], ws=ws)
+
+    sweep()
+    flush_l2(l2)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    sweep()
+    e1.record()
+    torch.cuda.synchronize()
+    t_ms = e0.elapsed_time(e1)
+    st, bits = q.qlora_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({bits:#x}) in the stack sweep")
+    fl = sum(fwd_flops(m, n, k, r) + bwd_flops(m, n, k, r) for _, n, k, _, _ in lin)
+    qb = sum(quant_bytes(n, k) for _, n, k, _, _ in lin)
+    del lin
+    return {"weights": params, "linears": 224, "quantize_ms": round(q_ms, 3),
+            "quantize_GB/s": round(qb / (q_ms * 1e-3) / 1e9, 1), "fwd_bwd_ms": round(t_ms, 3),
+            "fwd_bwd_TFLOP": round(fl / 1e12, 2), "fwd_bwd_TFLOP/s": round(fl / (t_ms * 1e-3) / 1e12, 1),
+            "workload": "whole 7B-shaped stack, 32 x (q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008), "
+                        "4096 tokens, r=64, weights generated on the GPU per layer"}
+
+
 def cpu_baseline_sample(target_s=15.0):
     """Time the oracle (as it stands) on a bounded sample of the same step:
     quantize the full W, forward + backward for `tok` tokens (fp64)."""
@@ -559,6 +622,9 @@ def run_ours(args):
     merge_ms, mb = merge_timing(q, wl, l2)
     popt = paged_optimizer(q, wl, l2)
     sib = fused_siblings(q, device, l2)
+    stack = whole_stack(q, device, l2)
+    stack["fwd_bwd_frac_of_sustained_bf16"] = round(stack["fwd_bwd_TFLOP/s"] / peaks["bf16_tflops_sustained"], 4)
+    stack["quantize_frac_hbm"] = round(stack["quantize_GB/s"] / peaks["hbm_gbs"], 4)
 
     # decode GEMV steady state + single-call latency
     gemv_ms, gemv_lat_ms, _ = gemv_steady_state(q, device)
@@ -629,6 +695,7 @@ def run_ours(args):
                   "method": "median of 10 calls, L2 flushed before each"},
         "paged_optimizer": popt,
         "fused_siblings": sib,
+        "whole_stack": stack,
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},

@@ -317,8 +317,9 @@ def test_backward_requires_n_multiple_of_8(q):
 
 # --------------------------------------------------------------------------- full size (bench launch shape)
 
-def test_full_size_7b_mlp_fwd_bwd_sampled(q):
-    p = synth.MLP7B
+@pytest.mark.parametrize("p", [synth.MLP7B, synth.Problem("7b-mlp-down-4096x11008-m4096-r64", 4096, 11008, 4096, 64,
+                                                         16.0)], ids=lambda p: p.name)
+def test_full_size_7b_mlp_fwd_bwd_sampled(q, p):
     t = synth.make(p)
     o = _oracle_quant(t["w"])
     w_hat = _oracle_what(o).astype(np.float64)
