@@ -370,6 +370,45 @@ def test_full_size_65b_fwd_bwd_sampled(q, p):
     assert linear.rel_fro(_np(db), s * (dyn.T @ (xn @ an.T))) <= TOL
 
 
+def test_decode_in_cuda_graph_sees_new_inputs(q):
+    # the decode path chains x A^T and the GEMV with programmatic dependent
+    # launch through a shared workspace; replaying a captured graph with new x
+    # (and a second call on the same workspace) must give exactly the direct
+    # calls' results
+    n, k, r, alpha = 1024, 512, 16, 16.0
+    qw = q.qlora_quantize_nf4(synth.weight(n, k, seed=13).cuda())
+    a = synth.lora_a(r, k, seed=14).cuda()
+    b = (synth.lora_b(n, r, seed=15).float() * 30).to(torch.bfloat16).cuda()
+    for m in (1, 5, 16):
+        x1 = torch.empty((m, k), dtype=torch.bfloat16, device="cuda")
+        x2 = torch.empty((m, k), dtype=torch.bfloat16, device="cuda")
+        y1 = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+        y2 = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(q.qlora_workspace_bytes(m, n, k, r) + 256, dtype=torch.uint8, device="cuda")
+        st = torch.cuda.Stream()
+        st.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(st):
+            q.qlora_linear_fwd(qw, x1, a, b, alpha, y=y1, ws=ws, want_u=False, stream=st)
+        st.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            q.qlora_linear_fwd(qw, x1, a, b, alpha, y=y1, ws=ws, want_u=False, stream=st)
+            q.qlora_linear_fwd(qw, x2, a, b, alpha, y=y2, ws=ws, want_u=False, stream=st)
+        for trial in range(3):
+            x1.copy_(synth.tokens(m, k, seed=100 + trial))
+            x2.copy_(synth.tokens(m, k, seed=200 + trial))
+            torch.cuda.synchronize()
+            g.replay()
+            torch.cuda.synchronize()
+            r1, _ = q.qlora_linear_fwd(qw, x1, a, b, alpha)
+            r2, _ = q.qlora_linear_fwd(qw, x2, a, b, alpha)
+            torch.cuda.synchronize()
+            assert torch.equal(y1.view(torch.int16), r1.view(torch.int16))
+            assert torch.equal(y2.view(torch.int16), r2.view(torch.int16))
+        del g
+    assert q.qlora_device_status() == (0, 0)
+
+
 def test_full_size_decode_gemv(q):
     p = synth.DECODE
     t = synth.make(p)
