@@ -48,7 +48,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # from one ncu capture, and a digest of the sources that build those kernels
 # at capture time. If any of them has changed since, the figure no longer
 # describes the kernel that runs and the roofline's traffic is reported null.
-FWD_TRAFFIC = {"bytes": 166318336, "sources_sha256": "513d96eb7ea1f3f4bcf58a79cb8e152b283431690616e47882f47736f5119334",
+FWD_TRAFFIC = {"bytes": 165788160, "sources_sha256": "58641100e1011491ae9fb950c0847f681e2382a31925957f3888036641214b0d",
                "profile": "profiles/qlora_linear_fwd_bwd_7b_mlp_dram.md"}
 FWD_SOURCES = ["api.cu", "tc_pair.cu", "tc_gemm.cu", "kernels.h", "ptx.cuh", "nf4_dev.cuh", "tc_common.cuh"]
 
@@ -462,6 +462,54 @@ def fused_siblings(q, device, l2, reps=5):
     return out
 
 
+def gemm_schedule(q, device, l2, reps=5):
+    """The pair GEMMs' schedule on the 65B-shaped projections (gate/up 22016x8192
+    and down 8192x22016, 4096 tokens, r=64): forward + backward under the
+    automatic rule (stream-K for these reductions of >= 128 k-tiles) against
+    forced data-parallel; median of `reps` calls, L2 flushed before each."""
+    out = {}
+    for p in (synth.GATE65B, synth.DOWN65B):
+        t = synth.make(p, seed=90)
+        qw = q.qlora_quantize_nf4(t["w"].to(device))
+        x, a, b, dy = (t[k_].to(device) for k_ in ("x", "a", "b", "dy"))
+        del t
+        y = torch.empty((p.m, p.n), dtype=torch.bfloat16, device=device)
+        u = torch.empty((p.m, p.r), dtype=torch.bfloat16, device=device)
+        dx = torch.empty((p.m, p.k), dtype=torch.bfloat16, device=device)
+        da = torch.empty((p.r, p.k), dtype=torch.float32, device=device)
+        db = torch.empty((p.n, p.r), dtype=torch.float32, device=device)
+        ws = torch.empty(q.qlora_workspace_bytes(p.m, p.n, p.k, p.r) + 256, dtype=torch.uint8, device=device)
+        res = {}
+        for name, mode in (("auto", q.SCHED_AUTO), ("data_parallel", q.SCHED_DATA_PARALLEL)):
+            q.qlora_set_gemm_schedule(mode)
+            try:
+                ts = {"fwd": [], "bwd": []}
+                for i in range(reps + 2):
+                    flush_l2(l2)
+                    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                    e[0].record()
+                    q.qlora_linear_fwd(qw, x, a, b, p.alpha, y=y, u=u, ws=ws)
+                    e[1].record()
+                    q.qlora_linear_bwd(qw, x, u, dy, a, b, p.alpha, dx=dx, da=da, db=db, ws=ws)
+                    e[2].record()
+                    torch.cuda.synchronize()
+                    if i >= 2:
+                        ts["fwd"].append(e[0].elapsed_time(e[1]))
+                        ts["bwd"].append(e[1].elapsed_time(e[2]))
+            finally:
+                q.qlora_set_gemm_schedule(q.SCHED_AUTO)
+            f_ms, b_ms = float(np.median(ts["fwd"])), float(np.median(ts["bwd"]))
+            res[name] = {"fwd_ms": round(f_ms, 4), "bwd_ms": round(b_ms, 4),
+                         "TFLOP/s": round((fwd_flops(p.m, p.n, p.k, p.r) + bwd_flops(p.m, p.n, p.k, p.r))
+                                          / ((f_ms + b_ms) * 1e-3) / 1e12, 1)}
+        res["speedup"] = round((res["data_parallel"]["fwd_ms"] + res["data_parallel"]["bwd_ms"])
+                               / (res["auto"]["fwd_ms"] + res["auto"]["bwd_ms"]), 3)
+        out[p.name] = res
+        del qw, x, a, b, dy, y, u, dx, da, db, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 def whole_stack(q, device, l2):
     """The whole 7B-shaped stack: 32 layers of q, k, v, o (4096x4096), gate,
     up (11008x4096) and down (4096x11008), 6,476,005,376 weights ~ N(0, 0.02).
@@ -622,6 +670,7 @@ def run_ours(args):
     merge_ms, mb = merge_timing(q, wl, l2)
     popt = paged_optimizer(q, wl, l2)
     sib = fused_siblings(q, device, l2)
+    sched = gemm_schedule(q, device, l2)
     stack = whole_stack(q, device, l2)
     stack["fwd_bwd_frac_of_sustained_bf16"] = round(stack["fwd_bwd_TFLOP/s"] / peaks["bf16_tflops_sustained"], 4)
     stack["quantize_frac_hbm"] = round(stack["quantize_GB/s"] / peaks["hbm_gbs"], 4)
@@ -695,6 +744,7 @@ def run_ours(args):
                   "method": "median of 10 calls, L2 flushed before each"},
         "paged_optimizer": popt,
         "fused_siblings": sib,
+        "gemm_schedule": sched,
         "whole_stack": stack,
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),

@@ -12,7 +12,7 @@ Functions carry the C names:
     qlora_workspace_bytes, qlora_fwd_workspace_bytes, qlora_linear_fwd, qlora_linear_fwd_ex,
     qlora_linear_fwd_noalloc, qlora_linear_bwd, qlora_device_status, qlora_status_string, qlora_version,
     qlora_launch_count, qlora_selftest_wait_timeout, qlora_merge_lora, qlora_adamw_step, qlora_adamw_host,
-    qlora_adamw_paged
+    qlora_adamw_paged, qlora_set_gemm_schedule, qlora_get_gemm_schedule
 """
 
 import ctypes
@@ -25,8 +25,9 @@ __all__ = [
     "qlora_linear_bwd",
     "qlora_device_status", "qlora_status_string", "qlora_version", "qlora_launch_count",
     "qlora_selftest_wait_timeout", "qlora_merge_lora", "qlora_adamw_step", "qlora_adamw_host", "qlora_adamw_paged",
+    "qlora_set_gemm_schedule", "qlora_get_gemm_schedule",
     "AdamwParams",
-    "FWD_AUTO", "FWD_GEMM", "FWD_GEMV",
+    "FWD_AUTO", "FWD_GEMM", "FWD_GEMV", "SCHED_AUTO", "SCHED_DATA_PARALLEL", "SCHED_STREAM_K",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlora.so")
@@ -38,6 +39,7 @@ if not os.path.exists(LIB_PATH):
 lib = ctypes.CDLL(LIB_PATH)
 
 FWD_AUTO, FWD_GEMM, FWD_GEMV = 0, 1, 2
+SCHED_AUTO, SCHED_DATA_PARALLEL, SCHED_STREAM_K = 0, 1, 2
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGNMENT", 4: "WORKSPACE",
                 5: "UNSUPPORTED_DEVICE", 6: "CUDA", 7: "TIMEOUT"}
 
@@ -103,6 +105,10 @@ lib.qlora_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _vp]
 lib.qlora_selftest_wait_timeout.restype = ctypes.c_int
 lib.qlora_launch_count.argtypes = []
 lib.qlora_launch_count.restype = ctypes.c_uint64
+lib.qlora_set_gemm_schedule.argtypes = [ctypes.c_int32]
+lib.qlora_set_gemm_schedule.restype = ctypes.c_int
+lib.qlora_get_gemm_schedule.argtypes = []
+lib.qlora_get_gemm_schedule.restype = ctypes.c_int32
 
 
 class QloraError(RuntimeError):
@@ -140,6 +146,15 @@ def qlora_version():
 def qlora_launch_count():
     """Kernels launched by the library in this process so far."""
     return int(lib.qlora_launch_count())
+
+
+def qlora_set_gemm_schedule(mode):
+    """Process-wide schedule of the pair GEMMs: SCHED_AUTO, SCHED_DATA_PARALLEL or SCHED_STREAM_K."""
+    _check(lib.qlora_set_gemm_schedule(int(mode)), "qlora_set_gemm_schedule")
+
+
+def qlora_get_gemm_schedule():
+    return int(lib.qlora_get_gemm_schedule())
 
 
 def qlora_status_string(status):

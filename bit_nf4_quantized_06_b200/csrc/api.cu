@@ -254,13 +254,42 @@ SmallPlan plan_small(int64_t rows, int64_t ktiles, int32_t r64, int sms) {
   return p;
 }
 
+// Token groups of 256 per restored weight tile: two once there are more than
+// 256 tokens (each restored tile then feeds 512 tokens), else one.
+inline int pair_nh(int64_t m) { return m > 256 ? 2 : 1; }
+
+// Stream-K slots of the pair kernels: one fp32 [128 x 256 NH] partial per CTA
+// (at most one CTA per SM) and four flags per CTA.
+inline size_t sk_part_bytes(int64_t m, int sms) {
+  return static_cast<size_t>(sms) * 128 * 256 * pair_nh(m) * sizeof(float);
+}
+inline size_t sk_flag_bytes(int sms) { return static_cast<size_t>(sms) * 4 * sizeof(uint32_t); }
+
+// Pair tiles of the forward (features = d_out) or dX (features = d_in).
+inline int64_t pair_tiles(int64_t m, int64_t features) {
+  return cdiv(features, 256) * cdiv(m, 256 * pair_nh(m));
+}
+
+// GEMM schedule setting (qlora_sched_t) and the automatic rule: stream-K for
+// reductions of at least kSkMinKtiles k-tiles.
+std::atomic<int> g_sched{QLORA_SCHED_AUTO};
+constexpr int64_t kSkMinKtiles = 128;
+inline bool sk_wanted(int64_t kt_main, int mode) {
+  return mode == QLORA_SCHED_STREAM_K || (mode == QLORA_SCHED_AUTO && kt_main >= kSkMinKtiles);
+}
+
 struct WsPlan {
   size_t u_pad, v_pad, b_pad, part, total;
+  bool sk_ok;        // a pair GEMM of the call may use the stream-K schedule
+  size_t sk_total;   // total with room for the stream-K slots (>= total)
 };
 
 // Workspace layout: [u_pad][v_pad][b_pad][split partials], each 256-aligned.
-// The forward needs no v_pad and only the x A^T partials.
-WsPlan plan_ws(int64_t m, int64_t n, int64_t k, int32_t r, int sms, bool fwd_only) {
+// The forward needs no v_pad and only the x A^T partials. The pair kernels'
+// stream-K slots reuse the partials region (it is free while they run), which
+// grows to hold them in the sk_total plan: `total` is what a call needs,
+// `sk_total` what lets it use the stream-K schedule when that pays.
+WsPlan plan_ws(int64_t m, int64_t n, int64_t k, int32_t r, int sms, bool fwd_only, int mode) {
   const int32_t r64 = r64_of(r);
   WsPlan w{};
   w.u_pad = al256(static_cast<size_t>(m) * r64 * 2);
@@ -274,6 +303,12 @@ WsPlan plan_ws(int64_t m, int64_t n, int64_t k, int32_t r, int sms, bool fwd_onl
   }
   w.part = al256(part);
   w.total = w.u_pad + w.v_pad + w.b_pad + w.part + 256;
+  // the forward reduces over K, dX over N; slots only where stream-K may run
+  const int64_t tiles = std::max(sk_wanted(cdiv(k, 64), mode) ? pair_tiles(m, n) : int64_t(0),
+                                 fwd_only || !sk_wanted(cdiv(n, 64), mode) ? int64_t(0) : pair_tiles(m, k));
+  const size_t sk = al256(sk_part_bytes(m, sms)) + al256(sk_flag_bytes(sms));
+  w.sk_ok = m > kGemvMaxM && tiles > sms / 4;
+  w.sk_total = w.sk_ok ? w.total - w.part + std::max(w.part, sk) : w.total;
   return w;
 }
 
@@ -340,15 +375,16 @@ qlora_status_t launch_pair_nh(int pairs, cudaStream_t st, const CUtensorMap& b, 
   return launch_status();
 }
 
-// Token groups of 256 per restored weight tile: two once there are more than
-// 256 tokens (each restored tile then feeds 512 tokens), else one.
-inline int pair_nh(int64_t m) { return m > 256 ? 2 : 1; }
-
 // The output [m x features] bf16 (row stride p.ldo) is written through TMA
 // stores when its row stride is a multiple of 16 bytes.
+//
+// Stream-K: with `sk_region` (the workspace's partials region, holding at
+// least the slots and flags of sk_part_bytes / sk_flag_bytes) and a tile
+// count above the pair count that leaves the last wave partly idle, the
+// pairs split the work evenly (see k_tc_pair); the flags are zeroed first.
 template <int AS>
 qlora_status_t launch_pair(int pairs, int64_t m, cudaStream_t st, const CUtensorMap& b, const CUtensorMap& bl,
-                           const CUtensorMap& c, TcParams p) {
+                           const CUtensorMap& c, TcParams p, uint8_t* sk_region, int sms, int mode) {
   CUtensorMap o = zero_map();
   p.tma_out = 0;
   if (p.ldo % 8 == 0 && (reinterpret_cast<uintptr_t>(p.out) & 15u) == 0) {
@@ -357,11 +393,22 @@ qlora_status_t launch_pair(int pairs, int64_t m, cudaStream_t st, const CUtensor
       return QLORA_ERR_CUDA;
     p.tma_out = 1;
   }
-  if (pair_nh(m) == 2) {
-    p.tiles_cols = static_cast<int32_t>(cdiv(m, 512));
-    return launch_pair_nh<AS, 2>(pairs, st, b, bl, c, o, p);
+  p.tiles_cols = static_cast<int32_t>(cdiv(m, 256 * pair_nh(m)));
+  const int64_t tiles = static_cast<int64_t>(p.tiles_rows) * p.tiles_cols;
+  p.sk = 0;
+  p.sk_part = nullptr;
+  p.sk_flags = nullptr;
+  if (sk_region != nullptr && sk_wanted(p.kt_main, mode) && p.tma_out && pairs > 1 && 2 * pairs <= sms &&
+      tiles > pairs && tiles % pairs != 0) {
+    p.sk = 1;
+    p.sk_part = reinterpret_cast<float*>(sk_region);
+    p.sk_flags = reinterpret_cast<uint32_t*>(sk_region + al256(sk_part_bytes(m, sms)));
+    if (cudaMemsetAsync(p.sk_flags, 0, sk_flag_bytes(sms), st) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
   }
-  p.tiles_cols = static_cast<int32_t>(cdiv(m, 256));
+  if (pair_nh(m) == 2) return launch_pair_nh<AS, 2>(pairs, st, b, bl, c, o, p);
   return launch_pair_nh<AS, 1>(pairs, st, b, bl, c, o, p);
 }
 
@@ -427,7 +474,8 @@ qlora_status_t check_linear(const LinearArgs& a, int sms, bool fwd_only) {
   if (!std::isfinite(a.alpha)) return QLORA_ERR_INVALID_ARG;
   if (a.m == 0) return QLORA_OK;
   if (a.ws == nullptr || !aligned16(a.ws)) return a.ws == nullptr ? QLORA_ERR_WORKSPACE : QLORA_ERR_ALIGNMENT;
-  if (a.ws_bytes < plan_ws(a.m, a.q->n_out, a.q->k_in, a.r, sms, fwd_only).total) return QLORA_ERR_WORKSPACE;
+  if (a.ws_bytes < plan_ws(a.m, a.q->n_out, a.q->k_in, a.r, sms, fwd_only, QLORA_SCHED_DATA_PARALLEL).total)
+    return QLORA_ERR_WORKSPACE;
   return QLORA_OK;
 }
 
@@ -441,6 +489,15 @@ extern "C" {
 int32_t qlora_version(void) { return 100; }
 
 uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+qlora_status_t qlora_set_gemm_schedule(int32_t mode) {
+  if (mode != QLORA_SCHED_AUTO && mode != QLORA_SCHED_DATA_PARALLEL && mode != QLORA_SCHED_STREAM_K)
+    return QLORA_ERR_INVALID_ARG;
+  g_sched.store(mode);
+  return QLORA_OK;
+}
+
+int32_t qlora_get_gemm_schedule(void) { return g_sched.load(); }
 
 const char* qlora_status_string(qlora_status_t s) {
   switch (s) {
@@ -492,12 +549,12 @@ int current_sms() {
 
 size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r) {
   if (m < 0 || n_out <= 0 || k_in <= 0 || r < 1 || r > kMaxRank) return 0;
-  return plan_ws(std::max<int64_t>(m, 1), n_out, k_in, r, current_sms(), false).total;
+  return plan_ws(std::max<int64_t>(m, 1), n_out, k_in, r, current_sms(), false, g_sched.load()).sk_total;
 }
 
 size_t qlora_fwd_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r) {
   if (m < 0 || n_out <= 0 || k_in <= 0 || r < 1 || r > kMaxRank) return 0;
-  return plan_ws(std::max<int64_t>(m, 1), n_out, k_in, r, current_sms(), true).total;
+  return plan_ws(std::max<int64_t>(m, 1), n_out, k_in, r, current_sms(), true, QLORA_SCHED_DATA_PARALLEL).total;
 }
 
 qlora_status_t qlora_quantize_nf4(const void* w_bf16, const qlora_nf4_t* q, void* stream) {
@@ -559,7 +616,8 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
   const int64_t n = q->n_out, k = q->k_in;
   const int32_t r64 = r64_of(r);
   const float sc = alpha / static_cast<float>(r);
-  const WsPlan wp = plan_ws(m, n, k, r, sms, true);
+  const int mode = g_sched.load();
+  const WsPlan wp = plan_ws(m, n, k, r, sms, true, mode);
   uint8_t* wsb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
   __nv_bfloat16* u_pad = reinterpret_cast<__nv_bfloat16*>(wsb);
   __nv_bfloat16* b_pad = reinterpret_cast<__nv_bfloat16*>(wsb + wp.u_pad + wp.v_pad);
@@ -676,7 +734,9 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
   p.lora_r = (r % 8 != 0) ? r64 : r;
   p.out = y;
   p.ldo = n;
-  return launch_pair<A_DQ_K>(pairs, m, st, m_x_b, m_u, m_codes, p);
+  return launch_pair<A_DQ_K>(pairs, m, st, m_x_b, m_u, m_codes, p,
+                             wp.sk_ok && ws_bytes >= wp.sk_total ? reinterpret_cast<uint8_t*>(part) : nullptr, sms,
+                             mode);
 }
 
 qlora_status_t qlora_linear_fwd(const qlora_nf4_t* q, const void* x, int64_t m, const void* a, const void* b,
@@ -711,7 +771,8 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
   }
   const int32_t r64 = r64_of(r);
   const float sc = alpha / static_cast<float>(r);
-  const WsPlan wp = plan_ws(m, n, k, r, sms, false);
+  const int mode = g_sched.load();
+  const WsPlan wp = plan_ws(m, n, k, r, sms, false, mode);
   uint8_t* wsb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
   __nv_bfloat16* u_pad = reinterpret_cast<__nv_bfloat16*>(wsb);
   __nv_bfloat16* v_pad = reinterpret_cast<__nv_bfloat16*>(wsb + wp.u_pad);
@@ -790,7 +851,9 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
     p.lora_r = r;
     p.out = dx;
     p.ldo = k;
-    s = launch_pair<A_DQ_MN>(pairs, m, st, m_dy_b, m_v, m_codes, p);
+    s = launch_pair<A_DQ_MN>(pairs, m, st, m_dy_b, m_v, m_codes, p,
+                             wp.sk_ok && ws_bytes >= wp.sk_total ? reinterpret_cast<uint8_t*>(part) : nullptr, sms,
+                             mode);
     if (s != QLORA_OK) return s;
   }
 

@@ -108,6 +108,14 @@ struct TcParams {
   int64_t ldo;          // pair kernel: row stride of out [cols x ldo]; small kernel: slabs [split][rows_pad][ldo]
   int32_t rows_pad;     // small kernel: rows per split slab
   int32_t tma_out;      // pair kernel: write the output through TMA stores
+  // pair kernel, stream-K schedule (sk = 1; needs tma_out): equal ranges of
+  // the (tile, k-tile) space per CTA pair; a tile cut between two pairs goes
+  // through one fp32 partial slot per CTA, [128 x 256 NH] floats each, laid
+  // out [column / 4][row][4], and four ready flags per CTA (one per epilogue
+  // warp), zeroed before the launch
+  int32_t sk;
+  float* sk_part;
+  uint32_t* sk_flags;
 };
 
 // TMA-fed tcgen05 GEMM for the small LoRA products: persistent CTAs (at most

@@ -83,6 +83,34 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// ------------------------------------------------------------------ global flags
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded wait until *flag != 0 (acquire at GPU scope); on timeout (or when
+// another role already aborted) records `code` and returns false.
+__device__ __forceinline__ bool flag_wait(const uint32_t* flag, volatile int* abort_flag, unsigned code) {
+  if (ld_acquire_gpu(flag) != 0) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (ld_acquire_gpu(flag) != 0) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > QLORA_WAIT_LIMIT_NS) {
+      atomicOr(&g_dev_status, code);
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(100);
+  }
+}
+
 // ------------------------------------------------------------------ fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -33,6 +33,20 @@
 //   warps 2-9   restore: two groups of four warps take alternate k-tiles
 //   warps 10-13 epilogue: drain this CTA's 128 token rows
 //
+// Schedules. Data-parallel: pair q takes tiles q, q + npairs, ... . When the
+// tile count is not a multiple of the pair count the last wave leaves pairs
+// idle; the stream-K schedule (p.sk) keeps all but the last full wave
+// data-parallel (the pairs then run in step and share their input tiles in
+// L2) and cuts the flattened (tile, k-tile) space of the remaining tiles --
+// between one and two waves' worth -- into one equal contiguous range per
+// pair. A range that ends inside a tile computes that tile's first k-tiles
+// (HEAD) and stores the fp32 partial sums in its slot; the next pair, whose
+// range starts inside that tile, computes the remaining k-tiles (TAIL), waits
+// for the slot's flags, adds the partial sums in its epilogue and writes the
+// tile. A pair processes its HEAD first and its TAIL only once it has done at
+// least as many k-tiles as the HEAD it depends on (plus a margin), so the wait
+// is normally already over; the writer always has the lower pair index.
+//
 // Every wait is bounded; every TMA load fills only the issuing CTA's shared
 // memory; the MMA's completion reaches the odd CTA through a commit to its
 // barrier's cluster address.
@@ -44,6 +58,88 @@
 namespace qlora {
 
 using namespace tcd;
+
+namespace {
+
+enum { SEG_FULL = 0, SEG_HEAD = 1, SEG_TAIL = 2 };
+constexpr int kSkMargin = 4;   // k-tiles of slack between a HEAD's end and the TAIL that reads it
+
+// One piece of work of a CTA pair: k-tiles [k0, k1) of a tile.
+struct Seg {
+  int tile, k0, k1, kind;
+};
+
+// The work list of one CTA pair (see the schedules above).
+struct PairWork {
+  int nseg, items, kt, pair, npairs;
+  bool sk;
+  int dp;                   // stream-K: data-parallel tiles pair, pair + npairs, ... done first
+  int head_tile, head_k1;   // HEAD: k-tiles [0, head_k1) of head_tile (head_tile < 0: none)
+  int tail_tile, tail_k0;   // TAIL: k-tiles [tail_k0, kt) of tail_tile (tail_tile < 0: none)
+  int full0, nfull, nf_before;   // full tiles full0 .. full0 + nfull - 1; nf_before of them precede the TAIL
+};
+
+__device__ __forceinline__ PairWork make_work(int pair, int npairs, int ntiles, int kt, bool sk) {
+  PairWork w{};
+  w.kt = kt;
+  w.pair = pair;
+  w.npairs = npairs;
+  w.sk = sk;
+  w.head_tile = -1;
+  w.tail_tile = -1;
+  if (!sk) {
+    w.nseg = (ntiles - pair + npairs - 1) / npairs;
+    w.items = w.nseg * kt;
+    return w;
+  }
+  // all but the last full wave stay data-parallel; the rest (at least one
+  // wave) is split, so every range holds at least kt k-tiles: a tile is cut
+  // at most once, and the HEAD and TAIL of one range lie in different tiles
+  w.dp = ntiles / npairs - 1;
+  const int base = w.dp * npairs;
+  const int64_t total = static_cast<int64_t>(ntiles - base) * kt;
+  const int64_t s0 = static_cast<int64_t>(base) * kt + static_cast<int64_t>(pair) * total / npairs;
+  const int64_t e0 = static_cast<int64_t>(base) * kt + static_cast<int64_t>(pair + 1) * total / npairs;
+  const int a = static_cast<int>(s0 / kt), ka = static_cast<int>(s0 % kt);
+  const int b = static_cast<int>(e0 / kt), kb = static_cast<int>(e0 % kt);
+  w.items = static_cast<int>(e0 - s0) + w.dp * kt;
+  w.full0 = a;
+  if (ka > 0) {
+    w.tail_tile = a;
+    w.tail_k0 = ka;
+    w.full0 = a + 1;
+  }
+  if (kb > 0) {
+    w.head_tile = b;
+    w.head_k1 = kb;
+  }
+  w.nfull = b - w.full0;
+  int done = kb, nb = 0;
+  if (ka > 0)
+    while (nb < w.nfull && done + (kt - ka) < ka + kSkMargin) {
+      done += kt;
+      ++nb;
+    }
+  w.nf_before = nb;
+  w.nseg = w.dp + w.nfull + (ka > 0 ? 1 : 0) + (kb > 0 ? 1 : 0);
+  return w;
+}
+
+__device__ __forceinline__ Seg seg_at(const PairWork& w, int i) {
+  if (!w.sk || i < w.dp) return Seg{w.pair + i * w.npairs, 0, w.kt, SEG_FULL};
+  i -= w.dp;
+  if (w.head_tile >= 0) {
+    if (i == 0) return Seg{w.head_tile, 0, w.head_k1, SEG_HEAD};
+    --i;
+  }
+  if (w.tail_tile >= 0) {
+    if (i == w.nf_before) return Seg{w.tail_tile, w.tail_k0, w.kt, SEG_TAIL};
+    if (i > w.nf_before) --i;
+  }
+  return Seg{w.full0 + i, 0, w.kt, SEG_FULL};
+}
+
+}  // namespace
 
 template <int AS, int NH>
 __global__ void __launch_bounds__(448, 1)
@@ -89,6 +185,7 @@ __global__ void __launch_bounds__(448, 1)
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
   const int ntile_total = p.tiles_rows * p.tiles_cols;  // 256-feature x (256 NH)-token tiles
+  const PairWork work = make_work(pair, npairs, ntile_total, p.kt_main + p.kt_lora, p.sk != 0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -124,13 +221,13 @@ __global__ void __launch_bounds__(448, 1)
       tma_prefetch_desc(&tm_t);
       tma_prefetch_desc(&tm_codes);
       if (p.kt_lora > 0) tma_prefetch_desc(&tm_t_lora);
-      const int ntiles = p.kt_main + p.kt_lora;
       int it = 0;
       bool ok = true;
-      for (int tile = pair; ok && tile < ntile_total; tile += npairs) {
-        const int f0 = tile_feat(tile);
-        const int tok = tile_tok(tile) + 128 * static_cast<int>(rank);
-        for (int t = 0; t < ntiles; ++t, ++it) {
+      for (int i = 0; ok && i < work.nseg; ++i) {
+        const Seg sg = seg_at(work, i);
+        const int f0 = tile_feat(sg.tile);
+        const int tok = tile_tok(sg.tile) + 128 * static_cast<int>(rank);
+        for (int t = sg.k0; t < sg.k1; ++t, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait(bar_empty(s), ph ^ 1, abort_flag, QLORA_DEV_TIMEOUT_PRODUCER)) {
@@ -167,16 +264,16 @@ __global__ void __launch_bounds__(448, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (even CTA)
     if (leader && lane == 0) {
-      const int ntiles = p.kt_main + p.kt_lora;
-      int it = 0, tcount = 0;
+      int it = 0;
       bool ok = true;
-      for (int tile = pair; ok && tile < ntile_total; tile += npairs, ++tcount) {
-        const int b = tcount % NBUF;
-        const uint32_t aph = (tcount / NBUF) & 1;
+      for (int i = 0; ok && i < work.nseg; ++i) {
+        const Seg sg = seg_at(work, i);
+        const int b = i % NBUF;
+        const uint32_t aph = (i / NBUF) & 1;
         if (!mbar_wait(bar_acce(b), aph ^ 1, abort_flag, QLORA_DEV_TIMEOUT_MMA)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * TILE_COLS;
-        for (int t = 0; t < ntiles; ++t, ++it) {
+        for (int t = sg.k0; t < sg.k1; ++t, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait(bar_full(s), ph, abort_flag, QLORA_DEV_TIMEOUT_MMA) ||
@@ -194,7 +291,7 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
             for (int h = 0; h < NH; ++h) {
               const uint64_t dt = smem_desc_sw128(t_s + h * T_HALF + kk * 32, 16, 1024);
-              tc_mma_pair(d_tmem + h * 256, dt, dw, IDESC, (t > 0 || kk > 0) ? 1u : 0u);
+              tc_mma_pair(d_tmem + h * 256, dt, dw, IDESC, (t > sg.k0 || kk > 0) ? 1u : 0u);
             }
           }
           tc_commit_pair(bar_empty(s));
@@ -212,24 +309,29 @@ __global__ void __launch_bounds__(448, 1)
     // ---------------------------------------------------------------- restore
     const int grp = (warp - 2) >> 2;                 // 0: warps 2-5, 1: warps 6-9
     const int tid = threadIdx.x - 64 - 128 * grp;    // 0..127
-    const int ipt = p.kt_main + p.kt_lora;
-    const int my_tiles = (ntile_total - pair + npairs - 1) / npairs;
-    const int items = my_tiles * ipt;
+    const int items = work.items;
     const uint32_t slot0 = ring + grp * (PD * 128 * 8) + tid * 8;
 
-    // cursor over this group's items j = grp, grp + 2, ...: k-tile t of a
-    // tile whose restored slice starts at feature f0
+    // cursor over this group's items j = grp, grp + 2, ... of the pair's
+    // work list: k-tile t (< k1) of segment i, whose restored slice starts at
+    // feature f0
     struct Cursor {
-      int j, t, tile, f0;
+      int j, i, t, k1, f0;
+    };
+    auto settle = [&](Cursor& c) {
+      while (c.i < work.nseg && c.t >= c.k1) {
+        const int over = c.t - c.k1;
+        if (++c.i >= work.nseg) break;
+        const Seg sg = seg_at(work, c.i);
+        c.t = sg.k0 + over;
+        c.k1 = sg.k1;
+        c.f0 = tile_feat(sg.tile);
+      }
     };
     auto advance = [&](Cursor& c) {
       c.j += 2;
       c.t += 2;
-      while (c.t >= ipt) {
-        c.t -= ipt;
-        c.tile += npairs;
-        c.f0 = tile_feat(c.tile);
-      }
+      settle(c);
     };
     // this thread's weight block for k-tile t (-1 = padding)
     auto block_of = [&](int f0, int t) -> int64_t {
@@ -262,12 +364,11 @@ __global__ void __launch_bounds__(448, 1)
       cp_async_commit();
     };
 
-    Cursor cur{grp, grp, pair, 0};
-    cur.f0 = tile_feat(cur.tile);
-    while (cur.t >= ipt) {
-      cur.t -= ipt;
-      cur.tile += npairs;
-      cur.f0 = tile_feat(cur.tile);
+    Cursor cur{};
+    {
+      const Seg sg0 = seg_at(work, 0);
+      cur = Cursor{grp, 0, sg0.k0 + grp, sg0.k1, tile_feat(sg0.tile)};
+      settle(cur);
     }
     Cursor pre = cur;
 #pragma unroll 1
@@ -384,26 +485,76 @@ __global__ void __launch_bounds__(448, 1)
     const bool vec_ok = (p.ldo % 8) == 0;
     const uint32_t box = epi_stage + (warp - 10) * 2048;
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
-    int tcount = 0;
-    for (int tile = pair; tile < ntile_total; tile += npairs, ++tcount) {
-      const int b = tcount % NBUF;
-      const uint32_t aph = (tcount / NBUF) & 1;
+    // stream-K partial slots hold float4 (column / 4, row) at [column / 4][row]
+    const int prow = quarter * 32 + lane;
+    constexpr int NCH = TILE_COLS / 32;
+    for (int si = 0; si < work.nseg; ++si) {
+      const Seg sg = seg_at(work, si);
+      const int tile = sg.tile;
+      const int b = si % NBUF;
+      const uint32_t aph = (si / NBUF) & 1;
       bool ok = mbar_wait(bar_accf(b), aph, abort_flag, QLORA_DEV_TIMEOUT_EPI);
       if (!warp_all(ok)) break;
       tc_fence_after();
       const int f0 = (tile / p.tiles_cols) * 256;   // first feature of the pair's tile
       const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
       const uint32_t tbase = tmem_base + b * TILE_COLS + lane_base;
+      auto release_acc = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader)
+            mbar_arrive(bar_acce(b));
+          else
+            mbar_arrive_cluster(acce_even0 + 8u * b);
+        }
+      };
+      if (sg.kind == SEG_HEAD) {
+        // partial sums of the tile's first k-tiles -> this CTA's slot, then
+        // this warp's ready flag (release after every lane's stores)
+        float4* slot = reinterpret_cast<float4*>(p.sk_part + static_cast<size_t>(blockIdx.x) * (128 * TILE_COLS)) + prow;
+        auto store8 = [&](int ch, const uint32_t (&r)[32]) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            slot[(ch * 8 + v) * 128] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                   __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+        };
+        uint32_t ra[32], rb[32];
+        tmem_ld_32x32b_x32(tbase, ra);
+        tc_wait_ld();
+#pragma unroll 1
+        for (int ch = 0; ch < NCH; ch += 2) {
+          tmem_ld_32x32b_x32(tbase + (ch + 1) * 32, rb);
+          store8(ch, ra);
+          tc_wait_ld();
+          if (ch + 2 < NCH) tmem_ld_32x32b_x32(tbase + (ch + 2) * 32, ra);
+          store8(ch + 1, rb);
+          if (ch + 2 < NCH) tc_wait_ld();
+        }
+        release_acc();
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          st_release_gpu(p.sk_flags + blockIdx.x * 4 + quarter, 1u);
+        }
+        continue;
+      }
+      const float4* part = nullptr;   // TAIL: the previous pair's partial sums for these rows
+      if (sg.kind == SEG_TAIL) {
+        const int wslot = static_cast<int>(blockIdx.x) - 2;
+        int fok = 1;
+        if (lane == 0) fok = flag_wait(p.sk_flags + wslot * 4 + quarter, abort_flag, QLORA_DEV_TIMEOUT_EPI) ? 1 : 0;
+        if (!__shfl_sync(0xFFFFFFFFu, fok, 0)) break;
+        part = reinterpret_cast<const float4*>(p.sk_part + static_cast<size_t>(wslot) * (128 * TILE_COLS)) + prow;
+      }
       if (p.tma_out) {
-        constexpr int NCH = TILE_COLS / 32;
-        // one 32-column chunk: convert `r`, start loading chunk ch + 1 into
-        // `nx`, stage and store `r`
-        auto chunk = [&](int ch, uint32_t (&r)[32], uint32_t (&nx)[32]) {
-          uint32_t pk[16];
+        // tensor memory column c: token group c / 256, feature c % 256
+        auto pack = [&](const uint32_t (&r)[32], uint32_t (&pk)[16]) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-          // tensor memory column c: token group c / 256, feature c % 256
-          if (ch + 1 < NCH) tmem_ld_32x32b_x32(tbase + (ch + 1) * 32, nx);
+        };
+        // stage one converted 32 x 32 chunk in this warp's box and store it
+        auto emit = [&](int ch, const uint32_t (&pk)[16]) {
           if (lane == 0) bulk_wait_read_all();   // the previous store has read the box
           __syncwarp();
           const uint32_t row = box + lane * 64;
@@ -419,25 +570,63 @@ __global__ void __launch_bounds__(448, 1)
             tma_store_2d(&tm_out, box, f0 + (ch % 8) * 32, token0);
             bulk_commit();
           }
-          if (ch + 1 < NCH) tc_wait_ld();
         };
-        uint32_t ra[32], rb[32];
-        tmem_ld_32x32b_x32(tbase, ra);
-        tc_wait_ld();
+        if (part == nullptr) {
+          // chunk ch + 1 loads from tensor memory while chunk ch is staged
+          uint32_t ra[32], rb[32];
+          tmem_ld_32x32b_x32(tbase, ra);
+          tc_wait_ld();
 #pragma unroll 1
-        for (int ch = 0; ch < NCH; ch += 2) {
-          chunk(ch, ra, rb);
-          chunk(ch + 1, rb, ra);
+          for (int ch = 0; ch < NCH; ch += 2) {
+            {
+              uint32_t pk[16];
+              pack(ra, pk);
+              tmem_ld_32x32b_x32(tbase + (ch + 1) * 32, rb);
+              emit(ch, pk);
+              tc_wait_ld();
+            }
+            {
+              uint32_t pk[16];
+              pack(rb, pk);
+              if (ch + 2 < NCH) tmem_ld_32x32b_x32(tbase + (ch + 2) * 32, ra);
+              emit(ch + 1, pk);
+              if (ch + 2 < NCH) tc_wait_ld();
+            }
+          }
+        } else {
+          // TAIL: the partial sums are read two chunks ahead (they come from
+          // L2 or HBM); one tensor-memory buffer keeps the registers in bounds
+          float4 pa[8], pb[8];
+          auto load_part = [&](int ch, float4 (&pq)[8]) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) pq[v] = __ldcg(part + (ch * 8 + v) * 128);
+          };
+          auto tail_chunk = [&](int ch, float4 (&pq)[8]) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tbase + ch * 32, r);
+            tc_wait_ld();
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              r[4 * v] = __float_as_uint(__uint_as_float(r[4 * v]) + pq[v].x);
+              r[4 * v + 1] = __float_as_uint(__uint_as_float(r[4 * v + 1]) + pq[v].y);
+              r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) + pq[v].z);
+              r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) + pq[v].w);
+            }
+            if (ch + 2 < NCH) load_part(ch + 2, pq);
+            uint32_t pk[16];
+            pack(r, pk);
+            emit(ch, pk);
+          };
+          load_part(0, pa);
+          load_part(1, pb);
+#pragma unroll 1
+          for (int ch = 0; ch < NCH; ch += 2) {
+            tail_chunk(ch, pa);
+            tail_chunk(ch + 1, pb);
+          }
         }
         // every column of this accumulator has been read: release it now
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if (leader)
-            mbar_arrive(bar_acce(b));
-          else
-            mbar_arrive_cluster(acce_even0 + 8u * b);
-        }
+        release_acc();
       } else {
 #pragma unroll 1
         for (int h = 0; h < NH; ++h) {
@@ -473,14 +662,7 @@ __global__ void __launch_bounds__(448, 1)
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if (leader)
-            mbar_arrive(bar_acce(b));
-          else
-            mbar_arrive_cluster(acce_even0 + 8u * b);
-        }
+        release_acc();
       }
     }
     if (lane == 0) bulk_wait_all();   // stores complete before the CTA's shared memory goes away

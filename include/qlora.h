@@ -123,14 +123,18 @@ QLORA_API qlora_status_t qlora_quantize_nf4(const void *w_bf16, const qlora_nf4_
 /* Restore W_hat [N x K] bf16 (device) from q. Bit-exact. */
 QLORA_API qlora_status_t qlora_dequantize(const qlora_nf4_t *q, void *w_bf16_out, void *stream);
 
-/* Workspace bytes that qlora_linear_fwd / _bwd need for these sizes (an
- * upper bound that covers both calls and every forward path). 0 for
- * arguments out of range. The size depends on the SM count of the current
- * device: ask with the device current that the calls will run on. */
+/* Workspace bytes for qlora_linear_fwd / _bwd at these sizes: covers both
+ * calls, every forward path, and, where the GEMM schedule
+ * (qlora_set_gemm_schedule) would use stream-K, its fp32 partial slots (up to
+ * 256 KB per SM). 0 for arguments out of range. The size depends on the SM
+ * count of the current device and on the schedule setting: ask with the
+ * device current that the calls will run on. A smaller workspace, down to
+ * what qlora_fwd_workspace_bytes reports for the forward, is accepted; the
+ * GEMMs then run data-parallel. */
 QLORA_API size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r);
 
-/* Workspace bytes that qlora_linear_fwd alone needs (at most
- * qlora_workspace_bytes for the same sizes). */
+/* The least workspace that qlora_linear_fwd accepts for these sizes (at most
+ * qlora_workspace_bytes for the same sizes; without the stream-K slots). */
 QLORA_API size_t qlora_fwd_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r);
 
 /* Forward: y [m x N] = x W_hat^T + s (x A^T) B^T, bf16 out, fp32 accumulate.
@@ -263,6 +267,32 @@ QLORA_API qlora_status_t qlora_device_status(void *stream, uint32_t *bits);
  * Lets a caller check that its error handling sees a timed-out wait without
  * any GPU fault. */
 QLORA_API qlora_status_t qlora_selftest_wait_timeout(uint32_t limit_us, void *stream);
+
+/* Work schedule of the CTA-pair GEMMs (forward y and backward dX); one
+ * setting for the whole process, read once per call.
+ *   QLORA_SCHED_AUTO (default): stream-K when the GEMM's reduction runs over
+ *     at least 128 k-tiles of 64 (K >= 8192 for the forward, d_out >= 8192
+ *     for dX) and its output tiles do not divide evenly over the SM pairs;
+ *     otherwise data-parallel. Measured on B200: with shorter reductions the
+ *     pairs' lockstep reuse of the input tiles in L2 is worth more than a
+ *     balanced last wave; with longer ones stream-K is 5-13 % faster.
+ *   QLORA_SCHED_DATA_PARALLEL: always data-parallel (tile q, q + pairs, ...).
+ *   QLORA_SCHED_STREAM_K: stream-K whenever the tiles do not divide evenly.
+ * Stream-K: all but the last full wave of tiles stay data-parallel, the rest
+ * is cut into equal (tile, k-tile) ranges, one per SM pair, and a tile cut
+ * between two pairs is finished from an fp32 partial passed through the
+ * workspace. It needs the workspace size that qlora_workspace_bytes reports
+ * under the same setting, and an output row stride that is a multiple of 8
+ * elements; otherwise the call runs data-parallel. Both schedules give the
+ * same results up to the order of fp32 additions. QLORA_ERR_INVALID_ARG for
+ * an unknown mode. */
+typedef enum {
+  QLORA_SCHED_AUTO = 0,
+  QLORA_SCHED_DATA_PARALLEL = 1,
+  QLORA_SCHED_STREAM_K = 2
+} qlora_sched_t;
+QLORA_API qlora_status_t qlora_set_gemm_schedule(int32_t mode);
+QLORA_API int32_t qlora_get_gemm_schedule(void);
 
 /* Static description of a status code. */
 QLORA_API const char *qlora_status_string(qlora_status_t s);

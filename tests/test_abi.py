@@ -120,3 +120,28 @@ def test_nf4_bytes_without_double_quantization(q):
     assert q.lib.qlora_dequantize(ctypes.byref(s), ctypes.c_void_p(16), None) == 1
     s = q.Nf4Struct(512, 512, 64, 0, 16, 0, 16)             # no scale codes needed without DQ
     assert q.lib.qlora_dequantize(ctypes.byref(s), None, None) == 1   # (null output still rejected)
+
+
+def test_gemm_schedule_setting(q):
+    assert q.qlora_get_gemm_schedule() == q.SCHED_AUTO
+    with pytest.raises(q.QloraError):
+        q.qlora_set_gemm_schedule(3)
+    assert q.qlora_get_gemm_schedule() == q.SCHED_AUTO
+    try:
+        # 4096 tokens, 4096 x 4096: reductions of 64 k-tiles, data-parallel under the automatic rule;
+        # forcing stream-K adds the partial slots (one fp32 [128 x 512] per SM) to the workspace
+        auto = q.qlora_workspace_bytes(4096, 4096, 4096, 64)
+        q.qlora_set_gemm_schedule(q.SCHED_STREAM_K)
+        forced = q.qlora_workspace_bytes(4096, 4096, 4096, 64)
+        assert forced >= auto + 128 * 512 * 4 * 32
+        q.qlora_set_gemm_schedule(q.SCHED_DATA_PARALLEL)
+        assert q.qlora_workspace_bytes(4096, 4096, 4096, 64) == auto
+        # reductions of >= 128 k-tiles (d_in 8192 forward, d_out 22016 for dX) use the slots by default
+        q.qlora_set_gemm_schedule(q.SCHED_AUTO)
+        assert q.qlora_workspace_bytes(4096, 22016, 8192, 64) > q.qlora_fwd_workspace_bytes(4096, 22016, 8192, 64) + 128 * 512 * 4 * 32
+        # the forward's least workspace never includes them
+        for mode in (q.SCHED_AUTO, q.SCHED_STREAM_K, q.SCHED_DATA_PARALLEL):
+            q.qlora_set_gemm_schedule(mode)
+            assert q.qlora_fwd_workspace_bytes(4096, 4096, 4096, 64) < forced
+    finally:
+        q.qlora_set_gemm_schedule(q.SCHED_AUTO)
