@@ -45,7 +45,7 @@ struct Tables {
   float mid[16];
   double cut[16];
   float cell_m[33];
-  uint32_t cell_info[33];
+  float cell_below[33];
 };
 
 const Tables& tables() {
@@ -82,7 +82,7 @@ const Tables& tables() {
         else if (r.mid[j] <= hi) cand = j;
       }
       r.cell_m[c] = cand >= 0 ? r.mid[cand] : 4.0f;
-      r.cell_info[c] = static_cast<uint32_t>(below) | (static_cast<uint32_t>(cand >= 0 ? cand : 15) << 8);
+      r.cell_below[c] = static_cast<float>(below);
     }
     return r;
   }();
@@ -567,7 +567,7 @@ qlora_status_t qlora_quantize_nf4(const void* w_bf16, const qlora_nf4_t* q, void
   QuantParams qp{};
   std::memcpy(qp.cut, tables().cut, sizeof(qp.cut));
   std::memcpy(qp.cell_m, tables().cell_m, sizeof(qp.cell_m));
-  std::memcpy(qp.cell_info, tables().cell_info, sizeof(qp.cell_info));
+  std::memcpy(qp.cell_below, tables().cell_below, sizeof(qp.cell_below));
   qp.dq = q->dq_group == kGroup ? 1 : 0;
   const int64_t groups = cdiv(nb, kGroup);
   if (groups > 0x7FFFFFFF) return QLORA_ERR_SHAPE;

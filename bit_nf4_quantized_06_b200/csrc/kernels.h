@@ -21,15 +21,15 @@ struct QuantParams {
   // Cell table of the encoder: cell c (0..32) holds the quotients x with
   // rint(16 x + 16) == c, widened by twice the guard below; cell_m[c] is the
   // one level midpoint m_j inside the widened cell (4.0 if there is none) and
-  // cell_info[c] packs (number of midpoints below the widened cell) | (j << 8).
+  // cell_below[c] the number of midpoints below the widened cell (a float).
   // A cell is 1/16 wide and the midpoints are more than 0.08 apart.
   float cell_m[33];
-  uint32_t cell_info[33];
+  float cell_below[33];
 };
-// |fl32(w * fl32(1/s)) - fl32(w / s)| <= 3.0001 * 2^-24 for |w| <= s; a
-// quotient farther than this guard from the candidate midpoint is decided
-// without the exact test.
-constexpr float kEncodeGuard = 4e-7f;
+// |fl32(w * r) - fl32(w / s)| < 3.4e-7 for |w| <= s, a normal s below 2^126
+// and r within 2 ulp of 1/s; a quotient farther than this guard from the
+// candidate midpoint is decided without the exact test.
+constexpr float kEncodeGuard = 5e-7f;
 
 struct DequantParams {
   float cb[16];   // the 16 fp32 levels

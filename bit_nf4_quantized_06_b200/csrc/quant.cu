@@ -30,16 +30,35 @@ __device__ unsigned int g_dev_status = 0;
 
 namespace {
 
+// Reciprocal by the hardware approximation (within 2 ulp for the normal
+// scales below 2^126 that reach it; the encoder's guard covers that error).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// Shared-memory load at a byte address; volatile keeps it after the barrier
+// that publishes the tables.
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t abs_bits_max(uint4 v) {
   // bf16 magnitudes compare like unsigned integers once the sign is cleared
-  uint32_t m = 0;
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    m = max(m, w[i] & 0x7FFFu);
-    m = max(m, (w[i] >> 16) & 0x7FFFu);
-  }
-  return m;
+  // (a NaN's pattern is above infinity's); both halves at once
+  uint32_t m = vmax_u16x2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+  m = vmax_u16x2(m, v.z & 0x7FFF7FFFu);
+  m = vmax_u16x2(m, v.w & 0x7FFF7FFFu);
+  return max(m & 0xFFFFu, m >> 16);
 }
 
 // Exact code of one weight by the division-free test: for a bf16 weight w
@@ -64,23 +83,28 @@ __device__ __noinline__ uint32_t exact_code(float w, float s, const double* cut)
 
 // One CTA of 256 threads per double-quantization group (see the file comment).
 //
-// Encode by cells: with r = fl32(1 / s), the quotient x' = fl32(w * r) lies
-// within 3.0001 * 2^-24 of fl32(w / s) for |w| <= s. Its cell
-// c = rint(16 x' + 16) (0..32, one fused multiply-add around a large
-// constant) selects a table entry holding the number of level midpoints
-// below the cell and the one midpoint m inside it (a cell is narrower than
-// the gaps between midpoints), so q = below + [x' > m] -- exactly the count
-// #{j : fl32(w / s) > m_j} whenever |x' - m| exceeds the guard. The two
-// 33-word tables sit in shared memory, one word per bank, so the lookups
-// never conflict. The rare weights within the guard of a midpoint, and
-// blocks whose scale is subnormal (1/s may overflow), take the exact test
-// above.
+// Encode by cells: with r the hardware reciprocal of s (within 2 ulp of 1 / s
+// for a normal s below 2^126), the quotient x' = fl32(w * r) lies within
+// 2^-22 + 2^-24 + 2^-25 < 3.4e-7 of fl32(w / s) for |w| <= s. Its cell c = rint(16 x' + 16) (0..32, one fused multiply-add
+// around a large constant) selects the one level midpoint m inside the cell
+// (a cell is narrower than the gaps between midpoints) and the number of
+// midpoints below it, so q = below + [x' > m] -- exactly the count
+// #{j : fl32(w / s) > m_j} whenever |x' - m| exceeds the guard. The work runs
+// on the floating-point pipe: [x' > m] is a saturated product
+// sat(d * 2^100) of d = x' - m (0 or 1), the near-midpoint test the sum over
+// the chunk of sat(G^2 - d^2) (positive when some |d| < G), and the eight
+// codes are packed into the 32-bit word by exact float multiply-adds
+// (integers below 2^16) read back through the 2^23 offset. The two 33-word
+// tables sit one word per bank, so the lookups never conflict; each is read
+// at 4 bits(t) + constant, t the cell's float. Chunks with a
+// quotient within the guard of a midpoint take the exact test above for
+// those weights; blocks whose scale is zero, subnormal, at least 2^126 or not
+// finite take it (or the value the definition gives) for every weight.
 __global__ void __launch_bounds__(256, 3) k_quantize_nf4(const uint4* __restrict__ w,
                                                       int64_t nb, uint32_t* __restrict__ codes,
                                                       uint8_t* __restrict__ q2,
                                                       float* __restrict__ smax, QuantParams qp) {
-  __shared__ float s_cm[33];
-  __shared__ uint32_t s_ci[33];
+  __shared__ float s_tab[66];     // [0, 33): the midpoint in each cell; [33, 66): midpoints below it
   __shared__ double s_cut[16];
   __shared__ uint32_t s_wmax[8];
   const int tid = threadIdx.x;
@@ -96,8 +120,8 @@ __global__ void __launch_bounds__(256, 3) k_quantize_nf4(const uint4* __restrict
     v[i] = (bi < nblk) ? __ldcs(w + chunk0 + tid + 256 * i) : make_uint4(0, 0, 0, 0);
   }
   if (tid < 33) {
-    s_cm[tid] = qp.cell_m[tid];
-    s_ci[tid] = qp.cell_info[tid];
+    s_tab[tid] = qp.cell_m[tid];
+    s_tab[33 + tid] = qp.cell_below[tid];
   }
   if (tid < 16) s_cut[tid] = qp.cut[tid];
 
@@ -120,79 +144,93 @@ __global__ void __launch_bounds__(256, 3) k_quantize_nf4(const uint4* __restrict
 #pragma unroll
   for (int i = 1; i < 8; ++i) gmax = max(gmax, s_wmax[i]);
   const float s_max = __uint_as_float(gmax << 16);
+  // per-block outputs: the eight lanes of a block group each take one of
+  // the group's eight blocks, (tid >> 3) + 32 * (tid & 7)
+  const int sub = tid & 7;
+  uint32_t my_am = am[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) my_am = (sub == i) ? am[i] : my_am;
+  const int my_bi = (tid >> 3) + 32 * sub;
   if (!qp.dq) {
     // 4.5-bit format: the block scale itself is stored (exact: a bf16 magnitude)
-    if ((tid & 7) == 0) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int bi = (tid >> 3) + 32 * i;
-        if (bi < nblk) smax[b0 + bi] = __uint_as_float(am[i] << 16);
+    if (my_bi < nblk) smax[b0 + my_bi] = __uint_as_float(my_am << 16);
+  } else {
+    if (tid == 0) smax[g] = s_max;
+    if (my_bi < nblk) {
+      uint32_t code = 0;
+      if (s_max != 0.0f) {
+        const float ratio = __fdiv_rn(256.0f * __uint_as_float(my_am << 16), s_max);
+        code = static_cast<uint32_t>(min(255, __float2int_rn(ratio)));
       }
-    }
-  } else if (tid == 0) {
-    smax[g] = s_max;
-  }
-
-  if (qp.dq && (tid & 7) == 0) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int bi = (tid >> 3) + 32 * i;
-      if (bi < nblk) {
-        uint32_t code = 0;
-        if (s_max != 0.0f) {
-          const float sb = __uint_as_float(am[i] << 16);
-          const float ratio = __fdiv_rn(256.0f * sb, s_max);
-          code = static_cast<uint32_t>(min(255, __float2int_rn(ratio)));
-        }
-        q2[b0 + bi] = static_cast<uint8_t>(code);
-      }
+      q2[b0 + my_bi] = static_cast<uint8_t>(code);
     }
   }
 
   constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: the integer part lands in the low mantissa bits
+  // shared address of cell c's midpoint is 4 * bits(t) + tab_base, t = 16 x + 16 + kMagic
+  const uint32_t tab_base = smem_u32(s_tab) - __float_as_uint(kMagic) * 4u;
+  constexpr float kGuard2 = kEncodeGuard * kEncodeGuard;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int bi = (tid >> 3) + 32 * i;
     if (bi < nblk) {
       const uint32_t a = am[i];
       const float sb = __uint_as_float(a << 16);
-      const bool zero = (a == 0);
-      const bool tiny = (a < 0x0080u);     // zero or subnormal scale
-      const float r = tiny ? 0.0f : __frcp_rn(sb);
+      // zero, subnormal, >= 2^126 (1/s subnormal), infinite or NaN scale
+      const bool edge = (a < 0x0080u) || (a >= 0x7E80u);
       const uint32_t ww[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-      uint32_t qv[8];
-      bool any_amb = false;
+      uint32_t word = 0;
+      bool slow = edge;
+      if (!edge) {
+        const float r = rcp_approx(sb);
+        float qf[8];
+        float amb = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        // element e of the chunk: bf16 pair e/2 holds element 2k in its low half
-        const float we = (e & 1) ? __uint_as_float(ww[e >> 1] & 0xFFFF0000u) : __uint_as_float(ww[e >> 1] << 16);
-        const float x = __fmul_rn(we, r);
-        const float t = fmaf(x, 16.0f, 16.0f + kMagic);
-        const uint32_t c = min(__float_as_uint(t) - __float_as_uint(kMagic), 32u);
-        const float d = __fsub_rn(x, s_cm[c]);
-        qv[e] = (s_ci[c] & 0xFFu) + (d > 0.0f ? 1u : 0u);
-        any_amb |= !(fabsf(d) > kEncodeGuard);
+        for (int e = 0; e < 8; ++e) {
+          // element e of the chunk: bf16 pair e/2 holds element 2k in its low half
+          const float we = (e & 1) ? __uint_as_float(ww[e >> 1] & 0xFFFF0000u) : __uint_as_float(ww[e >> 1] << 16);
+          const float x = __fmul_rn(we, r);
+          const float t = fmaf(x, 16.0f, 16.0f + kMagic);   // cell 0..32: |x| <= 1 + 2^-21
+          const uint32_t addr = __float_as_uint(t) * 4u + tab_base;
+          const float d = __fsub_rn(x, lds_f32(addr));
+          qf[e] = __fadd_rn(lds_f32(addr + 132u), __saturatef(__fmul_rn(d, 0x1p100f)));
+          amb = __fadd_rn(amb, __saturatef(fmaf(-d, d, kGuard2)));
+        }
+        if (amb > 0.0f) {
+          slow = true;
+        } else {
+          // byte j holds element 2j in its high nibble: word = lo + 2^16 hi
+          const float lo = __fadd_rn(fmaf(qf[2], 4096.0f, fmaf(qf[3], 256.0f, fmaf(qf[0], 16.0f, qf[1]))), 8388608.0f);
+          const float hi = __fadd_rn(fmaf(qf[6], 4096.0f, fmaf(qf[7], 256.0f, fmaf(qf[4], 16.0f, qf[5]))), 8388608.0f);
+          word = __float_as_uint(hi) * 65536u + __float_as_uint(lo) - 0x4B000000u;
+        }
       }
-      if (tiny || any_amb) {
-        // rare: redo the weights near a midpoint (or the whole block) exactly
+      if (slow) {
+        // rare: the exact test for the weights near a midpoint, or the whole block
+        const float r = edge ? 0.0f : rcp_approx(sb);
 #pragma unroll 1
         for (int e = 0; e < 8; ++e) {
           const float we = (e & 1) ? __uint_as_float(ww[e >> 1] & 0xFFFF0000u) : __uint_as_float(ww[e >> 1] << 16);
-          if (zero) {
-            qv[e] = 7u;
-          } else if (tiny) {
-            qv[e] = exact_code(we, sb, s_cut);
+          uint32_t q;
+          if (a == 0) {
+            q = 7u;                                    // s = 0 stores level 7
+          } else if (a >= 0x7F80u) {
+            // s = inf: fl32(w / s) = +-0 for finite w (7 midpoints below 0); NaN otherwise,
+            // which the definition orders above every midpoint
+            q = (a == 0x7F80u && (__float_as_uint(we) & 0x7F800000u) != 0x7F800000u) ? 7u : 15u;
+          } else if (edge) {
+            q = exact_code(we, sb, s_cut);
           } else {
             const float x = __fmul_rn(we, r);
             const float t = fmaf(x, 16.0f, 16.0f + kMagic);
-            const uint32_t c = min(__float_as_uint(t) - __float_as_uint(kMagic), 32u);
-            if (!(fabsf(__fsub_rn(x, s_cm[c])) > kEncodeGuard)) qv[e] = exact_code(we, sb, s_cut);
+            const uint32_t addr = __float_as_uint(t) * 4u + tab_base;
+            const float d = __fsub_rn(x, lds_f32(addr));
+            q = static_cast<uint32_t>(lds_f32(addr + 132u)) + (d > 0.0f ? 1u : 0u);
+            if (!(fabsf(d) > kEncodeGuard)) q = exact_code(we, sb, s_cut);
           }
+          word |= ((e & 1) ? q : (q << 4)) << (8 * (e >> 1));
         }
       }
-      uint32_t word = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) word |= ((qv[2 * j] << 4) | qv[2 * j + 1]) << (8 * j);
       codes[chunk0 + tid + 256 * i] = word;
     }
   }

@@ -130,6 +130,33 @@ def test_quantize_near_midpoints_bit_exact(q):
     assert np.array_equal(qn.absmax.cpu().numpy().view(np.uint32), o["absmax"].view(np.uint32))
 
 
+def test_quantize_nonfinite_and_huge_scales(q):
+    """Blocks whose scale the fast encoder does not take: +-inf and NaN weights
+    (s = inf: finite weights give fl32(w / s) = +-0, level 7; non-finite ones
+    a NaN quotient, which the definition's count orders above every midpoint:
+    15), and finite scales of at least 2^126 (1/s subnormal)."""
+    rng = np.random.default_rng(9)
+    w = (rng.standard_normal((16, 4096)) * 0.02).astype(np.float32)
+    w[0, 5] = np.inf
+    w[0, 70] = np.nan
+    w[0, 200] = -np.inf
+    w[0, 256:320] = rng.uniform(-1, 1, 64) * 2.0 ** 126
+    w[0, 256] = 2.0 ** 126
+    w[0, 320:384] = rng.uniform(-1, 1, 64) * 3.3e38
+    w[0, 320] = -3.3e38
+    w[5, 0:64] = rng.uniform(-1, 1, 64) * 3.3e38       # a finite group whose s_max is near the bf16 maximum
+    w[5, 0] = 3.3e38
+    w = obf16.round_to_bf16(w.ravel()).reshape(w.shape)
+    with np.errstate(all="ignore"):
+        o = nf4.quantize(w)
+    qw = q.qlora_quantize_nf4(torch.from_numpy(w).to(torch.bfloat16).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(qw.codes.cpu().numpy(), o["codes"].ravel())
+    # group 0 holds the NaN block (s_max NaN); the other groups are finite
+    assert np.array_equal(qw.scale_codes.cpu().numpy()[256:], o["q2"][256:])
+    assert np.array_equal(qw.absmax.cpu().numpy().view(np.uint32)[1:], o["smax"][1:].view(np.uint32))
+
+
 def test_quantize_full_size_7b_mlp(q):
     p = synth.MLP7B
     w = synth.weight(p.n, p.k)
