@@ -375,6 +375,24 @@ qlora_status_t launch_pair_nh(int pairs, cudaStream_t st, const CUtensorMap& b, 
   return launch_status();
 }
 
+// Features per tile of a data-parallel forward: of the widths 256, 240, ...,
+// 128 (multiples of 16: each CTA of a pair restores half, in 8-row swizzle
+// atoms) the one that needs the fewest features per pair over all waves,
+// ceil(tiles / pairs) * width, i.e. the one whose last wave is fullest; ties
+// go to the wider tile.
+int32_t pick_feat_n(int64_t features, int64_t tiles_cols, int pairs) {
+  int32_t best = 256;
+  int64_t best_cost = cdiv(cdiv(features, 256) * tiles_cols, pairs) * 256;
+  for (int32_t fn = 240; fn >= 128; fn -= 16) {
+    const int64_t cost = cdiv(cdiv(features, fn) * tiles_cols, pairs) * fn;
+    if (cost < best_cost) {
+      best = fn;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
 // The output [m x features] bf16 (row stride p.ldo) is written through TMA
 // stores when its row stride is a multiple of 16 bytes.
 //
@@ -394,6 +412,8 @@ qlora_status_t launch_pair(int pairs, int64_t m, cudaStream_t st, const CUtensor
     p.tma_out = 1;
   }
   p.tiles_cols = static_cast<int32_t>(cdiv(m, 256 * pair_nh(m)));
+  p.feat_n = 256;
+  p.tiles_rows = static_cast<int32_t>(cdiv(p.rows, 256));
   const int64_t tiles = static_cast<int64_t>(p.tiles_rows) * p.tiles_cols;
   p.sk = 0;
   p.sk_part = nullptr;
@@ -407,6 +427,10 @@ qlora_status_t launch_pair(int pairs, int64_t m, cudaStream_t st, const CUtensor
       cudaGetLastError();
       return QLORA_ERR_CUDA;
     }
+  }
+  if (AS == A_DQ_K && !p.sk && pairs > 0) {
+    p.feat_n = pick_feat_n(p.rows, p.tiles_cols, pairs);
+    p.tiles_rows = static_cast<int32_t>(cdiv(p.rows, p.feat_n));
   }
   if (pair_nh(m) == 2) return launch_pair_nh<AS, 2>(pairs, st, b, bl, c, o, p);
   return launch_pair_nh<AS, 1>(pairs, st, b, bl, c, o, p);

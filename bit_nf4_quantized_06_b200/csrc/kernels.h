@@ -116,6 +116,10 @@ struct TcParams {
   int32_t sk;
   float* sk_part;
   uint32_t* sk_flags;
+  // pair kernel: features per tile (the MMA's N), a multiple of 16 in
+  // [128, 256]; below 256 only for the forward (its restore takes any
+  // feature offset; dX slices must stay 64-aligned)
+  int32_t feat_n;
 };
 
 // TMA-fed tcgen05 GEMM for the small LoRA products: persistent CTAs (at most

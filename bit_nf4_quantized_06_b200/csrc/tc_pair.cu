@@ -1,14 +1,19 @@
 // Fused NF4-restore + tcgen05 GEMM on CTA pairs (cta_group::2), sm_100a.
 //
-// A cluster of two CTAs computes a (256 NH) tokens x 256 features tile of the
+// A cluster of two CTAs computes a (256 NH) tokens x FN features tile of the
 // output (y for the forward, dX for the backward), accumulating in fp32 in
 // tensor memory with tokens on the tensor-memory lanes:
 //
-//   D_h[256 tokens x 256 features] += T_h[256 x 64] * W[256 x 64]^T   per k-tile, h < NH
+//   D_h[256 tokens x FN features] += T_h[256 x 64] * W[FN x 64]^T   per k-tile, h < NH
+//
+// FN = 256, or for the data-parallel forward a narrower multiple of 16 that
+// fills the last wave better (11008 features: 46 tiles of 240 instead of 43
+// of 256, 4.97 waves of 74 pairs instead of 4.65); each CTA then restores
+// FN / 2 features (its 128 restore rows past them are ignored by the MMA).
 //
 // T_h is a 256-token slice of the input (x or dY), loaded by TMA, 128 tokens
 // per CTA. W is the 256-feature slice of the restored weight: CTA r restores
-// features [128 r, 128 r + 128) from the packed codes into the 128-byte
+// features [FN/2 r, FN/2 r + 128) from the packed codes into the 128-byte
 // swizzled layout the tensor core reads (K-major for the forward, MN-major
 // for dX, whose reduction runs along d_out while the 4-bit blocks run along
 // d_in). The even CTA issues the pair MMAs, which read both CTAs' shared
@@ -153,7 +158,8 @@ __global__ void __launch_bounds__(448, 1)
   constexpr uint32_t T_BYTES = NH * T_HALF;
   constexpr uint32_t C_BYTES = 4096;         // packed codes for the 128 features
   constexpr uint32_t STAGE_BYTES = W_BYTES + T_BYTES + C_BYTES;
-  constexpr uint32_t IDESC = idesc_bf16_f32(256, 256, false, W_MN);
+  const int FN = p.feat_n;                   // features per tile (multiple of 16, 128..256)
+  const uint32_t idesc = idesc_bf16_f32(256, FN, false, W_MN);
   constexpr uint32_t TILE_COLS = 256 * NH;   // accumulator columns per tile
   constexpr int NBUF = (NH == 1) ? 2 : 1;    // accumulator buffers (double-buffered when they fit)
   constexpr uint32_t TMEM_ALLOC = 512;
@@ -212,7 +218,7 @@ __global__ void __launch_bounds__(448, 1)
   const uint32_t tmem_base = *tmem_holder;
 
   // tile -> first feature of this CTA's restored slice, first token of the tile
-  auto tile_feat = [&](int tile) { return (tile / p.tiles_cols) * 256 + 128 * static_cast<int>(rank); };
+  auto tile_feat = [&](int tile) { return (tile / p.tiles_cols) * FN + (FN >> 1) * static_cast<int>(rank); };
   auto tile_tok = [&](int tile) { return (tile % p.tiles_cols) * static_cast<int>(TILE_COLS); };
 
   if (warp == 0) {
@@ -291,7 +297,7 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
             for (int h = 0; h < NH; ++h) {
               const uint64_t dt = smem_desc_sw128(t_s + h * T_HALF + kk * 32, 16, 1024);
-              tc_mma_pair(d_tmem + h * 256, dt, dw, IDESC, (t > sg.k0 || kk > 0) ? 1u : 0u);
+              tc_mma_pair(d_tmem + h * 256, dt, dw, idesc, (t > sg.k0 || kk > 0) ? 1u : 0u);
             }
           }
           tc_commit_pair(bar_empty(s));
@@ -496,7 +502,7 @@ __global__ void __launch_bounds__(448, 1)
       bool ok = mbar_wait(bar_accf(b), aph, abort_flag, QLORA_DEV_TIMEOUT_EPI);
       if (!warp_all(ok)) break;
       tc_fence_after();
-      const int f0 = (tile / p.tiles_cols) * 256;   // first feature of the pair's tile
+      const int f0 = (tile / p.tiles_cols) * FN;    // first feature of the pair's tile
       const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
       const uint32_t tbase = tmem_base + b * TILE_COLS + lane_base;
       auto release_acc = [&]() {
@@ -553,8 +559,28 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
         };
-        // stage one converted 32 x 32 chunk in this warp's box and store it
+        // stage one converted 32 x 32 chunk in this warp's box and store it;
+        // a chunk half inside the tile (FN % 32 == 16) goes out as two
+        // 16-byte stores per row, a chunk past it not at all
         auto emit = [&](int ch, const uint32_t (&pk)[16]) {
+          const int valid = FN - (ch % 8) * 32;
+          if (valid < 32) {
+            const int token = tile_tok(tile) + 256 * (ch / 8) + 128 * static_cast<int>(rank) + quarter * 32 + lane;
+            const int fc = f0 + (ch % 8) * 32;
+            if (valid > 0 && token < p.cols) {
+              __nv_bfloat16* orow = out + static_cast<int64_t>(token) * p.ldo + fc;
+              if (fc + 16 <= p.rows) {
+                reinterpret_cast<uint4*>(orow)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                reinterpret_cast<uint4*>(orow)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  if (fc + i < p.rows)
+                    reinterpret_cast<uint16_t*>(orow)[i] = static_cast<uint16_t>(pk[i >> 1] >> (16 * (i & 1)));
+              }
+            }
+            return;
+          }
           if (lane == 0) bulk_wait_read_all();   // the previous store has read the box
           __syncwarp();
           const uint32_t row = box + lane * 64;
@@ -640,11 +666,12 @@ __global__ void __launch_bounds__(448, 1)
             tmem_ld_32x32b_x32(taddr + ch * 32 + 32, r1);
             tc_wait_ld();
             if (token < p.cols) {
+              const int lim = min(p.rows, f0 + FN);   // features of this tile
 #pragma unroll
               for (int half = 0; half < 2; ++half) {
                 const uint32_t* rr = half ? r1 : r0;
                 const int fc = f0 + (ch + half) * 32;
-                if (vec_ok && fc + 32 <= p.rows) {
+                if (vec_ok && fc + 32 <= lim) {
                   uint4* dst = reinterpret_cast<uint4*>(orow + fc);
 #pragma unroll
                   for (int v = 0; v < 4; ++v) {
@@ -656,7 +683,7 @@ __global__ void __launch_bounds__(448, 1)
                 } else {
 #pragma unroll
                   for (int i = 0; i < 32; ++i)
-                    if (fc + i < p.rows) orow[fc + i] = __float2bfloat16_rn(__uint_as_float(rr[i]));
+                    if (fc + i < lim) orow[fc + i] = __float2bfloat16_rn(__uint_as_float(rr[i]));
                 }
               }
             }

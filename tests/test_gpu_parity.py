@@ -247,6 +247,38 @@ def test_forward_gemm_restores_w_exactly(q):
     assert np.array_equal(_bits(y).T, nf4.dequantize_bits(o["codes"], o["q2"], o["smax"]))
 
 
+def test_forward_narrow_tiles_restore_w_exactly(q):
+    # 4096 tokens over 11008 features: the data-parallel forward takes tiles of
+    # 240 features (46 x 8 tiles fill 74 pairs' five waves); x = I, B = 0 gives
+    # W_hat^T bit for bit, so every tile boundary and the 16-column tail
+    # chunk of each tile land where they should
+    n, k, r = 11008, 4096, 16
+    w = synth.weight(n, k, seed=31)
+    o = _oracle_quant(w)
+    qw = q.qlora_quantize_nf4(w.cuda())
+    x = torch.eye(k, dtype=torch.bfloat16, device="cuda")
+    a = synth.lora_a(r, k).cuda()
+    b = torch.zeros((n, r), dtype=torch.bfloat16, device="cuda")
+    y, _ = q.qlora_linear_fwd_ex(qw, x, a, b, 16.0, path=q.FWD_GEMM)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(y).T, nf4.dequantize_bits(o["codes"], o["q2"], o["smax"]))
+
+
+@pytest.mark.parametrize("n,k,m,r", [(4000, 192, 4096, 16), (11008, 128, 4096, 64), (12288, 64, 1000, 8)])
+def test_forward_narrow_tiles_parity(q, n, k, m, r):
+    # feature tiles of 224, 240 and 176 with ragged last tiles and token tails
+    alpha = 16.0
+    t = _problem(n, k, m, r, seed=n + m)
+    o = _oracle_quant(t["w"])
+    w_hat = _oracle_what(o)
+    y_ref, u_ref = linear.forward(_np(t["x"]), w_hat, _np(t["a"]), _np(t["b"]), alpha / r)
+    qw = q.qlora_quantize_nf4(t["w"].cuda())
+    y, u = q.qlora_linear_fwd_ex(qw, t["x"].cuda(), t["a"].cuda(), t["b"].cuda(), alpha, path=q.FWD_GEMM)
+    torch.cuda.synchronize()
+    assert linear.rel_fro(_np(y), y_ref) <= TOL
+    assert linear.rel_fro(_np(u), (alpha / r) * u_ref) <= TOL
+
+
 def test_forward_gemv_restores_w_exactly(q):
     n, k, r = 256, 512, 8
     w = synth.weight(n, k, seed=6)
