@@ -1,6 +1,6 @@
 """Run one library call on a named synthetic workload, for profilers.
 
-    python -m bit_nf4_quantized_06_b200.profile_case --op fwd --workload 7b-mlp --iters 3
+    python -m bit_nf4_quantized_06_b200.profile_case --op fwd --workload 7b-mlp --iters 3 [--schedule auto|dp|sk]
 
 Ops: quantize, dequantize, fwd (tensor-core path), bwd, gemv (decode path),
 merge (LoRA merge for export), adamw (adapter optimizer step, states on device).
@@ -35,7 +35,10 @@ def main(argv=None):
     ap.add_argument("--op", choices=["quantize", "dequantize", "fwd", "bwd", "gemv", "merge", "adamw"], required=True)
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="7b-mlp")
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--schedule", choices=["auto", "dp", "sk"], default="auto",
+                    help="GEMM schedule (qlora_set_gemm_schedule): automatic, data-parallel or stream-K")
     a = ap.parse_args(argv)
+    q.qlora_set_gemm_schedule({"auto": q.SCHED_AUTO, "dp": q.SCHED_DATA_PARALLEL, "sk": q.SCHED_STREAM_K}[a.schedule])
     p = WORKLOADS[a.workload]
     torch.cuda.set_device(0)
     t = synth.make(synth.Problem(p.name, p.n, p.k, p.m, p.r, p.alpha, p.outliers, True))
