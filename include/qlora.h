@@ -269,7 +269,10 @@ QLORA_API qlora_status_t qlora_device_status(void *stream, uint32_t *bits);
 QLORA_API qlora_status_t qlora_selftest_wait_timeout(uint32_t limit_us, void *stream);
 
 /* Work schedule of the CTA-pair GEMMs (forward y and backward dX); one
- * setting for the whole process, read once per call.
+ * setting for the whole process, read once per call. Not part of the method
+ * (the sources define what is computed, not how the work is split): a
+ * performance choice of this library that changes results only in the order
+ * of fp32 additions.
  *   QLORA_SCHED_AUTO (default): stream-K when the GEMM's reduction runs over
  *     at least 128 k-tiles of 64 (K >= 8192 for the forward, d_out >= 8192
  *     for dX) and its output tiles do not divide evenly over the SM pairs;
