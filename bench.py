@@ -518,12 +518,10 @@ def whole_stack(q, device, l2):
     bf16 copy freed. Then forward + backward of all 224 quantized linears at
     4096 tokens with r = 64 adapters, one event pair around the whole sweep."""
     m, r, alpha = 4096, 64, 16.0
-    gen = torch.Generator(device=device)
     lin, params, q_ms = [], 0, 0.0
     for layer in range(synth.STACK7B_LAYERS):
         for idx, (_, n, k) in enumerate(synth.STACK7B_LAYER):
-            gen.manual_seed(10_000 + 16 * layer + idx)
-            w = (torch.randn((n, k), generator=gen, device=device) * 0.02).to(torch.bfloat16)
+            w, a, b = synth.stack_linear(layer, idx, r=r, device=device)
             qw = q.NF4Weight(n, k, device=device)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
@@ -532,12 +530,9 @@ def whole_stack(q, device, l2):
             torch.cuda.synchronize()
             q_ms += e0.elapsed_time(e1)
             del w
-            a = (torch.rand((r, k), generator=gen, device=device) * 2 - 1).mul_(k ** -0.5).to(torch.bfloat16)
-            b = (torch.randn((n, r), generator=gen, device=device) * 0.01).to(torch.bfloat16)
             lin.append((qw, n, k, a, b))
             params += n * k
-    xs = {k: torch.randn((m, k), generator=gen, device=device).to(torch.bfloat16) for k in (4096, 11008)}
-    dys = {n: torch.randn((m, n), generator=gen, device=device).to(torch.bfloat16) for n in (4096, 11008)}
+    xs, dys = synth.stack_activations(m, device=device)
     ys = {n: torch.empty((m, n), dtype=torch.bfloat16, device=device) for n in (4096, 11008)}
     dxs = {k: torch.empty((m, k), dtype=torch.bfloat16, device=device) for k in (4096, 11008)}
     u = torch.empty((m, r), dtype=torch.bfloat16, device=device)

@@ -94,7 +94,8 @@ struct DevState {
   bool checked = false;
   bool ok = false;
   int sms = 148;
-  bool attrs = false;
+  bool attrs = false;      // kernel attributes set in context `ctx`
+  CUcontext ctx = nullptr;
   int pair_clusters = 0;   // CTA pairs of k_tc_pair that can be resident at once
 };
 std::mutex g_mu;
@@ -158,6 +159,41 @@ cudaError_t pair_clusters(int* out) {
   return (*out > 0) ? cudaSuccess : cudaErrorInvalidConfiguration;
 }
 
+}  // namespace
+
+// The calling thread's current CUDA context, made current by the runtime if
+// needed (cuCtxGetCurrent through the runtime's driver entry point, so the
+// library needs no link-time dependency on the driver library).
+CUcontext current_context() {
+  using Fn = CUresult (*)(CUcontext*);
+  static Fn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return static_cast<Fn>(nullptr);
+    }
+    return reinterpret_cast<Fn>(p);
+  }();
+  if (fn == nullptr) return nullptr;
+  CUcontext c = nullptr;
+  if (fn(&c) != CUDA_SUCCESS) return nullptr;
+  if (c == nullptr) {
+    // nothing has used the runtime on this thread yet: cudaSetDevice
+    // initialises the device's primary context and makes it current
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    if (fn(&c) != CUDA_SUCCESS) return nullptr;
+  }
+  return c;
+}
+
+namespace {
+
 qlora_status_t device_ready(int* sms_out, int* pairs_out = nullptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_CUDA;
@@ -171,6 +207,11 @@ qlora_status_t device_ready(int* sms_out, int* pairs_out = nullptr) {
     st.sms = prop.multiProcessorCount;
   }
   if (!st.ok) return QLORA_ERR_UNSUPPORTED_DEVICE;
+  // kernel attributes belong to the context: set them again in a new one
+  // (after cudaDeviceReset the runtime creates a new primary context)
+  CUcontext ctx = current_context();
+  if (ctx == nullptr) return QLORA_ERR_CUDA;
+  if (st.attrs && st.ctx != ctx) st.attrs = false;
   if (!st.attrs) {
     cudaError_t e = pair_clusters(&st.pair_clusters);
     if (e == cudaSuccess) e = set_small_attrs<64>();
@@ -182,11 +223,20 @@ qlora_status_t device_ready(int* sms_out, int* pairs_out = nullptr) {
                                static_cast<int>(merge_smem_bytes(kMaxRank)));
     if (e != cudaSuccess) return QLORA_ERR_CUDA;
     st.attrs = true;
+    st.ctx = ctx;
   }
   if (sms_out) *sms_out = st.sms;
   if (pairs_out) *pairs_out = st.pair_clusters;
   return QLORA_OK;
 }
+
+}  // namespace
+
+// The same device check every entry point runs first (see device_ready), for
+// the entry points defined in other files.
+int check_current_device_status() { return static_cast<int>(device_ready(nullptr)); }
+
+namespace {
 
 // ------------------------------------------------------------------ helpers
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -279,13 +329,15 @@ inline bool sk_wanted(int64_t kt_main, int mode) {
 }
 
 struct WsPlan {
-  size_t u_pad, v_pad, b_pad, part, total;
+  size_t u_pad, v_pad, b_pad, dy_pad, part, total;
   bool sk_ok;        // a pair GEMM of the call may use the stream-K schedule
   size_t sk_total;   // total with room for the stream-K slots (>= total)
 };
 
-// Workspace layout: [u_pad][v_pad][b_pad][split partials], each 256-aligned.
-// The forward needs no v_pad and only the x A^T partials. The pair kernels'
+// Workspace layout: [u_pad][v_pad][b_pad][dy_pad][split partials], each
+// 256-aligned. The forward needs no v_pad, no dy_pad and only the x A^T
+// partials. dy_pad holds dY with its rows padded to a multiple of 8 elements
+// when N % 8 != 0 (the TMA loads of dY need 16-byte row strides). The pair kernels'
 // stream-K slots reuse the partials region (it is free while they run), which
 // grows to hold them in the sk_total plan: `total` is what a call needs,
 // `sk_total` what lets it use the stream-K schedule when that pays.
@@ -295,6 +347,7 @@ WsPlan plan_ws(int64_t m, int64_t n, int64_t k, int32_t r, int sms, bool fwd_onl
   w.u_pad = al256(static_cast<size_t>(m) * r64 * 2);
   w.v_pad = fwd_only ? 0 : al256(static_cast<size_t>(m) * r64 * 2);
   w.b_pad = (r % 8 != 0) ? al256(static_cast<size_t>(n) * r64 * 2) : 0;
+  w.dy_pad = (!fwd_only && n % 8 != 0) ? al256(static_cast<size_t>(m) * rup(n, 8) * 2) : 0;
   size_t part = plan_small(m, cdiv(k, 64), r64, sms).part_bytes;  // x A^T
   if (!fwd_only) {
     part = std::max(part, plan_small(m, cdiv(n, 64), r64, sms).part_bytes);  // dY B
@@ -302,7 +355,7 @@ WsPlan plan_ws(int64_t m, int64_t n, int64_t k, int32_t r, int sms, bool fwd_onl
     part = std::max(part, plan_small(n, cdiv(m, 64), r64, sms).part_bytes);  // dB
   }
   w.part = al256(part);
-  w.total = w.u_pad + w.v_pad + w.b_pad + w.part + 256;
+  w.total = w.u_pad + w.v_pad + w.b_pad + w.dy_pad + w.part + 256;
   // the forward reduces over K, dX over N; slots only where stream-K may run
   const int64_t tiles = std::max(sk_wanted(cdiv(k, 64), mode) ? pair_tiles(m, n) : int64_t(0),
                                  fwd_only || !sk_wanted(cdiv(n, 64), mode) ? int64_t(0) : pair_tiles(m, k));
@@ -645,7 +698,7 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
   uint8_t* wsb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
   __nv_bfloat16* u_pad = reinterpret_cast<__nv_bfloat16*>(wsb);
   __nv_bfloat16* b_pad = reinterpret_cast<__nv_bfloat16*>(wsb + wp.u_pad + wp.v_pad);
-  float* part = reinterpret_cast<float*>(wsb + wp.u_pad + wp.v_pad + wp.b_pad);
+  float* part = reinterpret_cast<float*>(wsb + wp.u_pad + wp.v_pad + wp.b_pad + wp.dy_pad);
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
   const auto* ab = static_cast<const __nv_bfloat16*>(a);
   const auto* bb = static_cast<const __nv_bfloat16*>(b);
@@ -784,7 +837,6 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
       (dx && !aligned16(dx)) || (u && !aligned16(u)))
     return QLORA_ERR_ALIGNMENT;
   const int64_t n = q->n_out, k = q->k_in;
-  if (n % 8 != 0) return QLORA_ERR_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (m == 0) {
     // no tokens: the gradients are exactly zero
@@ -801,11 +853,20 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
   __nv_bfloat16* u_pad = reinterpret_cast<__nv_bfloat16*>(wsb);
   __nv_bfloat16* v_pad = reinterpret_cast<__nv_bfloat16*>(wsb + wp.u_pad);
   __nv_bfloat16* b_pad = reinterpret_cast<__nv_bfloat16*>(wsb + wp.u_pad + wp.v_pad);
-  float* part = reinterpret_cast<float*>(wsb + wp.u_pad + wp.v_pad + wp.b_pad);
+  __nv_bfloat16* dy_pad = reinterpret_cast<__nv_bfloat16*>(wsb + wp.u_pad + wp.v_pad + wp.b_pad);
+  float* part = reinterpret_cast<float*>(wsb + wp.u_pad + wp.v_pad + wp.b_pad + wp.dy_pad);
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
   const auto* ab = static_cast<const __nv_bfloat16*>(a);
   const auto* bb = static_cast<const __nv_bfloat16*>(b);
   const auto* dyb = static_cast<const __nv_bfloat16*>(dy);
+  // dY rows reach the tensor maps with a 16-byte stride: pad them when N % 8 != 0
+  const int64_t ldn = rup(n, 8);
+  if (ldn != n) {
+    k_pad_cols<<<static_cast<unsigned>(std::min<int64_t>(cdiv(m * ldn, 256), int64_t(sms) * 8)), 256, 0, st>>>(
+        dyb, dy_pad, m, static_cast<int32_t>(n), static_cast<int32_t>(ldn));
+    if ((s = launch_status()) != QLORA_OK) return s;
+    dyb = dy_pad;
+  }
   const __nv_bfloat16* b_use = bb;
   int64_t ldb = r;
   if (r % 8 != 0) {
@@ -839,7 +900,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
   // v' = bf16(s dY B): A = dY (K-major), B = B_lora seen MN-major, reduction over N
   {
     CUtensorMap m_dy_a, m_bmn;
-    if (!map_bf16(&m_dy_a, dyb, m, n, n, 128) || !map_bf16(&m_bmn, b_use, n, ldb == r ? r : r64, ldb, 64))
+    if (!map_bf16(&m_dy_a, dyb, m, n, ldn, 128) || !map_bf16(&m_bmn, b_use, n, ldb == r ? r : r64, ldb, 64))
       return QLORA_ERR_CUDA;
     s = lora_product<A_TMA_K, B_TMA_MN>(m_dy_a, m_bmn, m, n, r, sc, 0, v_pad, nullptr, nullptr, part, sms, st);
     if (s != QLORA_OK) return s;
@@ -849,7 +910,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
   // plus v' A_lora as extra k-tiles
   if (dx != nullptr) {
     CUtensorMap m_dy_b, m_v, m_codes;
-    if (!map_bf16(&m_dy_b, dyb, m, n, n, 128) || !map_bf16(&m_v, v_pad, m, r64, r64, 128) ||
+    if (!map_bf16(&m_dy_b, dyb, m, n, ldn, 128) || !map_bf16(&m_v, v_pad, m, r64, r64, 128) ||
         !map2d(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->codes, static_cast<uint64_t>(k / 2),
                static_cast<uint64_t>(n), static_cast<uint64_t>(k / 2), 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
       return QLORA_ERR_CUDA;
@@ -891,7 +952,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
   // dB [N x r] = dY^T u'  (A = dY seen MN-major, B = u' MN-major)
   {
     CUtensorMap m_dymn, m_umn;
-    if (!map_bf16(&m_dymn, dyb, m, n, n, 64) || !map_bf16(&m_umn, u_use, m, ldu == r ? r : r64, ldu, 64))
+    if (!map_bf16(&m_dymn, dyb, m, n, ldn, 64) || !map_bf16(&m_umn, u_use, m, ldu == r ? r : r64, ldu, 64))
       return QLORA_ERR_CUDA;
     s = lora_product<A_TMA_MN, B_TMA_MN>(m_dymn, m_umn, n, m, r, 1.0f, 1, nullptr, nullptr, db, part, sms, st);
     if (s != QLORA_OK) return s;

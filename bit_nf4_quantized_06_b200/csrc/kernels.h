@@ -218,6 +218,16 @@ inline size_t merge_smem_bytes(int r64) {
   return static_cast<size_t>(128) * (r64 + 8) * 2 + static_cast<size_t>(r64) * 136 * 2 + 128 * 132 * 4;
 }
 
+// Device check of the current device (sm_100, attributes set), as every entry
+// point runs it: QLORA_OK, QLORA_ERR_UNSUPPORTED_DEVICE or QLORA_ERR_CUDA
+// (values of qlora_status_t, returned as int to keep the ABI header out).
+int check_current_device_status();
+
+// The calling thread's current CUDA context (nullptr on failure). Entry
+// points call it after check_current_device_status, which has made the
+// runtime's primary context current.
+CUcontext current_context();
+
 // Zero-padded copy of a [rows x r] bf16 matrix into [rows x r64].
 __global__ void k_pad_cols(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
                            int64_t rows, int32_t r, int32_t r64);

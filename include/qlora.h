@@ -161,18 +161,26 @@ QLORA_API qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t *q, const void *x
  * way to hand over scratch memory: a runtime whose device memory all belongs
  * to its own pool, code running where a device allocation is forbidden or
  * would stall other work (cudaMalloc may synchronise the device), or a plain
- * C caller with no device allocator. This call computes exactly what
- * qlora_linear_fwd computes, with the same arguments minus ws/ws_bytes, and
- * uses instead one fixed device array of QLORA_NOALLOC_SCRATCH_BYTES owned by
- * the library. It allocates and frees nothing.
+ * C caller with no device allocator. This call takes the arguments of
+ * qlora_linear_fwd minus ws/ws_bytes and uses instead one fixed device array
+ * of QLORA_NOALLOC_SCRATCH_BYTES owned by the library. It allocates and
+ * frees nothing.
+ *   - Results: it is qlora_linear_fwd given that array as a workspace of
+ *     QLORA_NOALLOC_SCRATCH_BYTES bytes, and so bit-identical to
+ *     qlora_linear_fwd called with a caller workspace of that same size. The
+ *     array is too small for the stream-K slots, so the GEMM always runs the
+ *     data-parallel schedule; where qlora_linear_fwd with a larger
+ *     workspace would run stream-K (qlora_set_gemm_schedule), results agree
+ *     within the forward's tolerance, not bit for bit.
  *   - Problems whose qlora_fwd_workspace_bytes() exceeds the array are
  *     rejected with QLORA_ERR_WORKSPACE before anything is launched. Ask
  *     that function beforehand: the need follows the split plan and is not
  *     monotone in m. On a 148-SM B200 at r <= 64 every m up to 2,304 tokens
  *     fits for 4096 x 11008 and 8192 x 22016 weights of either orientation
  *     (up to 6,272 for 11008 x 4096 and 4096 x 4096); at r = 256 up to 384.
- *   - The first call on each device looks up the array's device address with
- *     that device current; make that first call before any stream capture.
+ *   - The first call on each device (and the first after a cudaDeviceReset)
+ *     looks up the array's device address with that device current; make
+ *     that first call before any stream capture.
  *   - Every call shares the one array and leaves its contents behind; no part
  *     of it needs to start at zero (each call writes all it reads). Calls
  *     that overlap on the GPU (other streams, other host threads) race on it:
@@ -184,7 +192,8 @@ QLORA_API qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t *q, const vo
 /* Backward: dX [m x K] bf16 (may be NULL to skip), dA [r x K] fp32 and
  * dB [N x r] fp32 (overwritten, not accumulated). u_bf16 is the u' that the
  * forward produced ([m x r], may be NULL: then it is recomputed). No gradient
- * into W. N % 8 == 0 is required here (dY rows are read by TMA). */
+ * into W. Any N: when N % 8 != 0 the call first copies dY into the workspace
+ * with its rows padded to a multiple of 8 (qlora_workspace_bytes counts it). */
 QLORA_API qlora_status_t qlora_linear_bwd(const qlora_nf4_t *q, const void *x_bf16, const void *u_bf16,
                                 const void *dy_bf16, int64_t m, const void *a_bf16,
                                 const void *b_bf16, int32_t r, float alpha, void *dx_bf16,

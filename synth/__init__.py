@@ -13,6 +13,10 @@ Distributions (one derived seed per tensor, base seed 0 by default):
     dY ~ N(0, 1)                   seed + 4
     outlier mask U(0,1) < 0.001    seed + 5   (entries of W scaled x20
                                                before the bf16 cast)
+
+The whole 7B-shaped stack (6.5 billion weights) is the exception: its
+tensors are drawn on the GPU with a device generator (stack_linear,
+stack_activations), deterministic for a given device type.
 """
 
 import math
@@ -90,6 +94,34 @@ STACK7B_LAYER = (
     ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008),
 )
 STACK7B_LAYERS = 32
+STACK7B_SEED = 10_000          # + 16 * layer + projection index
+STACK7B_ACT_SEED = 20_000      # activations and upstream gradients of the stack
+
+
+def stack_linear(layer, idx, r=64, device="cuda"):
+    """W [n, k], A [r, k], B [n, r] (bf16, on `device`) of projection `idx`
+    of `layer` in the 7B-shaped stack, drawn on the device from one
+    generator seeded STACK7B_SEED + 16 * layer + idx, in the order W, A, B:
+    W ~ N(0, 0.02), A ~ U(+-1/sqrt(k)), B ~ N(0, 0.01). Generated on the GPU
+    because the whole stack holds 6.5 billion weights."""
+    _, n, k = STACK7B_LAYER[idx]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(STACK7B_SEED + 16 * layer + idx)
+    w = (torch.randn((n, k), generator=gen, device=device) * 0.02).to(torch.bfloat16)
+    a = (torch.rand((r, k), generator=gen, device=device) * 2 - 1).mul_(k ** -0.5).to(torch.bfloat16)
+    b = (torch.randn((n, r), generator=gen, device=device) * 0.01).to(torch.bfloat16)
+    return w, a, b
+
+
+def stack_activations(m=4096, device="cuda"):
+    """Inputs x [m, k] for k in (4096, 11008) and upstream gradients dY [m, n]
+    for n in (4096, 11008) of the stack's linears (bf16, N(0, 1)), drawn on
+    the device from one generator seeded STACK7B_ACT_SEED."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(STACK7B_ACT_SEED)
+    xs = {k: torch.randn((m, k), generator=gen, device=device).to(torch.bfloat16) for k in (4096, 11008)}
+    dys = {n: torch.randn((m, n), generator=gen, device=device).to(torch.bfloat16) for n in (4096, 11008)}
+    return xs, dys
 
 
 def make(p: Problem, seed=0):

@@ -366,18 +366,72 @@ def test_backward_dx_restores_w_exactly(q):
     assert torch.count_nonzero(da).item() == 0        # B = 0 -> no gradient into A
 
 
-def test_backward_requires_n_multiple_of_8(q):
-    n, k, m, r = 100, 128, 16, 8
-    t = _problem(n, k, m, r)
+# d_out not a multiple of 8: the forward's output rows are not 16-byte
+# multiples, so its epilogue stores each row directly instead of through TMA
+# boxes; the backward copies dY into row-padded workspace first
+ODD_N_CASES = [
+    (1001, 512, 300, 16),
+    (37, 192, 64, 8),
+    (100, 128, 16, 8),       # 16 tokens through the GEMM path
+    (1001, 256, 700, 100),   # two token groups per tile, r not a multiple of 8
+]
+
+
+@pytest.mark.parametrize("n,k,m,r", ODD_N_CASES)
+def test_odd_d_out_forward_backward_parity(q, n, k, m, r):
+    alpha = 16.0
+    s = alpha / r
+    t = _problem(n, k, m, r, seed=5 * n + k + m)
+    o = _oracle_quant(t["w"])
+    w_hat = _oracle_what(o)
+    y_ref, u_ref = linear.forward(_np(t["x"]), w_hat, _np(t["a"]), _np(t["b"]), s)
+    dx_ref, da_ref, db_ref = linear.backward(_np(t["x"]), _np(t["dy"]), w_hat, _np(t["a"]), _np(t["b"]), s)
     qw = q.qlora_quantize_nf4(t["w"].cuda())
-    with pytest.raises(q.QloraError):
-        q.qlora_linear_bwd(qw, t["x"].cuda(), None, t["dy"].cuda(), t["a"].cuda(), t["b"].cuda(), 16.0)
+    x, a, b, dy = (t[k_].cuda() for k_ in ("x", "a", "b", "dy"))
+    y, u = q.qlora_linear_fwd_ex(qw, x, a, b, alpha, path=q.FWD_GEMM)
+    dx, da, db = q.qlora_linear_bwd(qw, x, u, dy, a, b, alpha)
+    torch.cuda.synchronize()
+    assert linear.rel_fro(_np(y), y_ref) <= TOL
+    assert linear.rel_fro(_np(u), s * u_ref) <= TOL
+    assert linear.rel_fro(_np(dx), dx_ref) <= TOL
+    assert linear.rel_fro(_np(da), da_ref) <= TOL
+    assert linear.rel_fro(_np(db), db_ref) <= TOL
+
+
+def test_odd_d_out_forward_restores_w_exactly(q):
+    # x = I, B = 0 through the direct-store epilogue: y = W_hat^T bit for bit
+    n, k, r = 1001, 192, 16
+    w = synth.weight(n, k, seed=9)
+    o = _oracle_quant(w)
+    qw = q.qlora_quantize_nf4(w.cuda())
+    x = torch.eye(k, dtype=torch.bfloat16)
+    b = torch.zeros((n, r), dtype=torch.bfloat16)
+    y, _ = q.qlora_linear_fwd_ex(qw, x.cuda(), synth.lora_a(r, k).cuda(), b.cuda(), 16.0, path=q.FWD_GEMM)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(y).T, nf4.dequantize_bits(o["codes"], o["q2"], o["smax"]))
+
+
+def test_odd_d_out_backward_dx_restores_w_exactly(q):
+    # dY = I (tokens = N rows) with N = 1001, B = 0: dX = W_hat bit for bit
+    # through the row-padded copy of dY
+    n, k, r = 1001, 256, 16
+    w = synth.weight(n, k, seed=10)
+    o = _oracle_quant(w)
+    qw = q.qlora_quantize_nf4(w.cuda())
+    dy = torch.eye(n, dtype=torch.bfloat16)
+    b = torch.zeros((n, r), dtype=torch.bfloat16)
+    dx, da, db = q.qlora_linear_bwd(qw, synth.tokens(n, k).cuda(), None, dy.cuda(), synth.lora_a(r, k).cuda(),
+                                    b.cuda(), 16.0)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(dx), nf4.dequantize_bits(o["codes"], o["q2"], o["smax"]))
 
 
 # --------------------------------------------------------------------------- full size (bench launch shape)
 
-@pytest.mark.parametrize("p", [synth.MLP7B, synth.Problem("7b-mlp-down-4096x11008-m4096-r64", 4096, 11008, 4096, 64,
-                                                         16.0)], ids=lambda p: p.name)
+@pytest.mark.parametrize("p", [synth.MLP7B,
+                               synth.Problem("7b-mlp-down-4096x11008-m4096-r64", 4096, 11008, 4096, 64, 16.0),
+                               synth.Problem("7b-attn-4096x4096-m4096-r64", 4096, 4096, 4096, 64, 16.0)],
+                         ids=lambda p: p.name)
 def test_full_size_7b_mlp_fwd_bwd_sampled(q, p):
     t = synth.make(p)
     o = _oracle_quant(t["w"])
