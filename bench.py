@@ -661,19 +661,21 @@ def run_ours(args):
     f_fl, b_fl = fwd_flops(p.m, p.n, p.k, p.r), bwd_flops(p.m, p.n, p.k, p.r)
     value = world * wl.flops / (step_ms * 1e-3) / 1e12
 
-    # LoRA merge for export and the paged adapter optimizer (outside the step)
-    merge_ms, mb = merge_timing(q, wl, l2)
-    popt = paged_optimizer(q, wl, l2)
-    sib = fused_siblings(q, device, l2)
-    sched = gemm_schedule(q, device, l2)
-    stack = whole_stack(q, device, l2)
-    stack["fwd_bwd_frac_of_sustained_bf16"] = round(stack["fwd_bwd_TFLOP/s"] / peaks["bf16_tflops_sustained"], 4)
-    stack["quantize_frac_hbm"] = round(stack["quantize_GB/s"] / peaks["hbm_gbs"], 4)
-
-    # decode GEMV steady state + single-call latency
-    gemv_ms, gemv_lat_ms, _ = gemv_steady_state(q, device)
-    gb = gemv_bytes(d.n, d.k, d.r)
-    gemv_gbs = gb / (gemv_ms * 1e-3) / 1e9
+    # single-GPU measurements outside the step (N = 1 only: every rank would
+    # repeat them on its own GPU)
+    extras = world == 1
+    if extras:
+        merge_ms, mb = merge_timing(q, wl, l2)
+        popt = paged_optimizer(q, wl, l2)
+        sib = fused_siblings(q, device, l2)
+        sched = gemm_schedule(q, device, l2)
+        stack = whole_stack(q, device, l2)
+        stack["fwd_bwd_frac_of_sustained_bf16"] = round(stack["fwd_bwd_TFLOP/s"] / peaks["bf16_tflops_sustained"], 4)
+        stack["quantize_frac_hbm"] = round(stack["quantize_GB/s"] / peaks["hbm_gbs"], 4)
+        # decode GEMV steady state + single-call latency
+        gemv_ms, gemv_lat_ms, _ = gemv_steady_state(q, device)
+        gb = gemv_bytes(d.n, d.k, d.r)
+        gemv_gbs = gb / (gemv_ms * 1e-3) / 1e9
 
     # end to end through host buffers: H2D of x, dY, W; D2H of dA, dB and the decode output
     e2e_ms = None
@@ -728,25 +730,26 @@ def run_ours(args):
             "bwd": {"ms": round(b_ms, 4), "TFLOP/s": round(b_ach, 1), "frac": round(b_ach / peak_t, 4)},
             "decode_in_step": {"ms": round(g_ms, 4)},
         },
-        "gemv": {"workload": d.name, "us_per_call_steady": round(gemv_ms * 1e3, 3),
-                 "us_single_call": round(gemv_lat_ms * 1e3, 3), "bytes_per_call": gb, "GB/s": round(gemv_gbs, 1),
-                 "frac_hbm": round(gemv_gbs / peaks["hbm_gbs"], 4), "peak_hbm_gbs": peaks["hbm_gbs"],
-                 "frac_vs_8tbs": round(gemv_gbs / 8000.0, 4),
-                 "method": "CUDA graph of 200 calls over 32 rotating packed weights (277 MB > 2x L2), x5 replays"},
-        "merge": {"workload": p.name + " LoRA merge for export, bf16(W_hat + s B A)", "ms": round(merge_ms, 4),
-                  "bytes": int(mb), "GB/s": round(mb / (merge_ms * 1e-3) / 1e9, 1),
-                  "frac_hbm": round(mb / (merge_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                  "method": "median of 10 calls, L2 flushed before each"},
-        "paged_optimizer": popt,
-        "fused_siblings": sib,
-        "gemm_schedule": sched,
-        "whole_stack": stack,
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": int(launches),
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
     }
+    if extras:
+        line["gemv"] = {"workload": d.name, "us_per_call_steady": round(gemv_ms * 1e3, 3),
+                        "us_single_call": round(gemv_lat_ms * 1e3, 3), "bytes_per_call": gb,
+                        "GB/s": round(gemv_gbs, 1), "frac_hbm": round(gemv_gbs / peaks["hbm_gbs"], 4),
+                        "peak_hbm_gbs": peaks["hbm_gbs"], "frac_vs_8tbs": round(gemv_gbs / 8000.0, 4),
+                        "method": "CUDA graph of 200 calls over 32 rotating packed weights (277 MB > 2x L2), x5 replays"}
+        line["merge"] = {"workload": p.name + " LoRA merge for export, bf16(W_hat + s B A)", "ms": round(merge_ms, 4),
+                         "bytes": int(mb), "GB/s": round(mb / (merge_ms * 1e-3) / 1e9, 1),
+                         "frac_hbm": round(mb / (merge_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                         "method": "median of 10 calls, L2 flushed before each"}
+        line["paged_optimizer"] = popt
+        line["fused_siblings"] = sib
+        line["gemm_schedule"] = sched
+        line["whole_stack"] = stack
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_sample()
     if world > 1:
@@ -809,6 +812,28 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def torchrun_command(n, script, argv, port):
+    """The command that starts `n` ranks of `script` on this node, one process
+    per GPU (rank i on GPU i through LOCAL_RANK), rendezvous on 127.0.0.1."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", "--master-port", str(port), script] + list(argv)
+
+
+def free_port():
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def spawn_ranks(n, script, argv, timeout_s=1800):
+    """Run `script` as `n` ranks under torch.distributed.run and return its exit
+    status (the ranks' JSON line is printed by rank 0). Used when the bench is
+    started with --gpus N > 1 outside a launcher."""
+    cmd = torchrun_command(n, script, argv, free_port())
+    return subprocess.call(["timeout", "-k", "60", str(timeout_s)] + cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -817,6 +842,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # data-parallel over N GPUs of this node: start N ranks of this script
+        sys.exit(spawn_ranks(args.gpus, os.path.abspath(__file__), sys.argv[1:]))
+    if "WORLD_SIZE" in os.environ and int(os.environ["WORLD_SIZE"]) != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={os.environ['WORLD_SIZE']}; the run uses WORLD_SIZE",
+              file=sys.stderr)
     if args.impl == "reference":
         args.steps = 3 if args.steps is None else args.steps
         args.warmup = 1 if args.warmup is None else args.warmup

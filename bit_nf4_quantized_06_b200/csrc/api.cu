@@ -372,6 +372,7 @@ qlora_status_t check_nf4(const qlora_nf4_t* q) {
   if (q->n_out <= 0 || q->k_in <= 0 || q->k_in % kBlock != 0) return QLORA_ERR_SHAPE;
   if (q->n_out > (int64_t(1) << 31) - 1 || q->k_in > (int64_t(1) << 31) - 1) return QLORA_ERR_SHAPE;
   if (!aligned16(q->codes)) return QLORA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(q->absmax) & 3u) != 0) return QLORA_ERR_ALIGNMENT;
   return QLORA_OK;
 }
 

@@ -182,3 +182,55 @@ def merge(w_hat, a, b, s):
             row.append(bf16_round_bits(Fraction(w_hat[i][c]) + sf * acc))
         out.append(row)
     return out
+
+
+def double_quantize_u8_255(scales, group=256):
+    """The 255-step unsigned scale code, one exact rounding per operation:
+    q2 = min(255, rint_even(fl32(fl32(255 s) / s_max))), s_hat = fl32(fl32(q2 s_max) / 255)."""
+    q2, smax_l, s_hat = [], [], []
+    for g0 in range(0, len(scales), group):
+        grp = scales[g0:g0 + group]
+        smax = max(grp)
+        smax_l.append(smax)
+        for s in grp:
+            if smax == 0:
+                q = 0
+            else:
+                ratio = f32_round(Fraction(f32_round(Fraction(255) * Fraction(s))) / Fraction(smax))
+                q = min(255, _rint_even(Fraction(ratio)))
+            q2.append(q)
+            s_hat.append(f32_round(Fraction(f32_round(Fraction(q) * Fraction(smax))) / 255))
+    return q2, smax_l, s_hat
+
+
+def double_quantize_s8_mid(scales, group=256):
+    """The signed mid-range scale code, one exact rounding per operation:
+    mid = fl32(fl32(lo + hi) / 2), half = fl32(fl32(hi - lo) / 2),
+    q2 = clamp(rint_even(fl32(fl32(127 fl32(s - mid)) / half)), -127, 127),
+    s_hat = fl32(mid + fl32(fl32(q2 half) / 127))."""
+    q2, gdata, s_hat = [], [], []
+    for g0 in range(0, len(scales), group):
+        grp = scales[g0:g0 + group]
+        lo, hi = min(grp), max(grp)
+        mid = f32_round(Fraction(f32_round(Fraction(lo) + Fraction(hi))) / 2)
+        half = f32_round(Fraction(f32_round(Fraction(hi) - Fraction(lo))) / 2)
+        gdata.append((mid, half))
+        for s in grp:
+            if half == 0:
+                q = 0
+            else:
+                t = f32_round(Fraction(s) - Fraction(mid))
+                ratio = f32_round(Fraction(f32_round(127 * Fraction(t))) / Fraction(half))
+                q = max(-127, min(127, _rint_even(Fraction(ratio))))
+            q2.append(q)
+            s_hat.append(f32_round(Fraction(mid) + Fraction(f32_round(Fraction(f32_round(Fraction(q) * Fraction(half))) / 127))))
+    return q2, gdata, s_hat
+
+
+def _rint_even(q):
+    """Round a rational to the nearest integer, ties to even."""
+    fl = q.numerator // q.denominator
+    rem = q - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return int(fl)

@@ -220,3 +220,123 @@ def max_level_gap(c=None):
 def normal_cdf(z):
     """Phi via math.erf, independent of NormalDist.inv_cdf (used by the pins)."""
     return 0.5 * (1.0 + math.erf(z / math.sqrt(2.0)))
+
+
+# --------------------------------------------------------------------------- scale-code variants
+#
+# The printed double quantization (reading 4) codes each block scale on the
+# unsigned grid s_max * q2 / 256. Two further codes of the 8-bit scale, both
+# readings of the same paragraph («QLoRA는 어떻게 65B 모델을 GPU 한 장에
+# 올렸나», § "메모리 회계: 세 겹의 최적화": 8-bit codes of the scales with a
+# 32-bit constant per group, error bounded by the grid step):
+#
+# "u8_255": the unsigned grid with 255 steps, so the top code is exact:
+#     q2    = min(255, rint_even(fl32(fl32(255 s) / s_max)))   (0 if s_max = 0)
+#     s_hat = fl32(fl32(q2 s_max) / 255)
+#   group data: s_max (one float32); error at most s_max / 510 (+ rounding).
+#
+# "s8_mid": a signed code centred on the group's mid-range, two float32
+#   constants per group:
+#     lo, hi = min s, max s over the group
+#     mid    = fl32(fl32(lo + hi) / 2),  half = fl32(fl32(hi - lo) / 2)
+#     q2     = clamp(rint_even(fl32(fl32(127 fl32(s - mid)) / half)), -127, 127)   (0 if half = 0)
+#     s_hat  = fl32(mid + fl32(fl32(q2 half) / 127))
+#   q2 stored as int8 (two's complement bytes); error at most half / 254
+#   (+ rounding), far below s_max / 256 when the group's scales are close.
+
+DQ_CODES = ("u8_256", "u8_255", "s8_mid")
+
+
+def group_data_floats(code):
+    """float32 constants stored per group of 256 block scales."""
+    return 2 if code == "s8_mid" else 1
+
+
+def double_quantize_code(absmax, code):
+    """Scale codes and group data of `code` (see above).
+
+    Returns (q2 uint8 [nb] (int8 bits for s8_mid), gdata float32 [ng] or [ng, 2]).
+    """
+    if code == "u8_256":
+        return double_quantize(absmax)
+    a = np.asarray(absmax, dtype=np.float32)
+    ng = n_groups(a.size)
+    g = np.arange(a.size) // DQ_GROUP
+    if code == "u8_255":
+        smax = group_smax(a)
+        sm = smax[g]
+        zero = sm == 0.0
+        with np.errstate(divide="ignore", invalid="ignore"):
+            ratio = ((np.float32(255.0) * a).astype(np.float32) / np.where(zero, np.float32(1.0), sm)).astype(np.float32)
+        q2 = np.minimum(np.float32(255.0), np.rint(ratio)).astype(np.uint8)
+        q2[zero] = 0
+        return q2, smax
+    if code == "s8_mid":
+        pad_hi = np.full(ng * DQ_GROUP, -np.inf, dtype=np.float32)
+        pad_lo = np.full(ng * DQ_GROUP, np.inf, dtype=np.float32)
+        pad_hi[: a.size] = a
+        pad_lo[: a.size] = a
+        hi = pad_hi.reshape(ng, DQ_GROUP).max(axis=1)
+        lo = pad_lo.reshape(ng, DQ_GROUP).min(axis=1)
+        mid = ((lo + hi).astype(np.float32) * np.float32(0.5)).astype(np.float32)
+        half = ((hi - lo).astype(np.float32) * np.float32(0.5)).astype(np.float32)
+        t = (a - mid[g]).astype(np.float32)
+        hz = half[g] == 0.0
+        with np.errstate(divide="ignore", invalid="ignore"):
+            ratio = ((np.float32(127.0) * t).astype(np.float32) / np.where(hz, np.float32(1.0), half[g])).astype(np.float32)
+        q = np.clip(np.rint(ratio), -127, 127).astype(np.int8)
+        q[hz] = 0
+        return q.view(np.uint8), np.stack([mid, half], axis=1).astype(np.float32)
+    raise ValueError(code)
+
+
+def restored_scale_code(q2, gdata, code):
+    """s_hat per block for `code` (float32 [nb])."""
+    if code == "u8_256":
+        return restored_scale(q2, gdata)
+    q2 = np.asarray(q2, dtype=np.uint8)
+    g = np.arange(q2.size) // DQ_GROUP
+    if code == "u8_255":
+        prod = (q2.astype(np.float32) * np.asarray(gdata, dtype=np.float32)[g]).astype(np.float32)
+        return (prod / np.float32(255.0)).astype(np.float32)
+    if code == "s8_mid":
+        gd = np.asarray(gdata, dtype=np.float32).reshape(-1, 2)
+        mid, half = gd[g, 0], gd[g, 1]
+        qs = q2.view(np.int8).astype(np.float32)
+        t = ((qs * half).astype(np.float32) / np.float32(127.0)).astype(np.float32)
+        return (mid + t).astype(np.float32)
+    raise ValueError(code)
+
+
+def quantize_code(w, code):
+    """Quantizer with scale code `code`: dict with codes, q2, gdata (and absmax, q for checking)."""
+    w = np.asarray(w, dtype=np.float32)
+    absmax = block_absmax(w)
+    q = encode(w, absmax)
+    q2, gdata = double_quantize_code(absmax, code)
+    return {"codes": pack(q), "q2": q2, "gdata": gdata, "absmax": absmax, "q": q}
+
+
+def dequantize_bits_code(codes, q2, gdata, code):
+    """Restored weights (bf16 bits, uint16 [N, K]) for scale code `code`:
+    w_hat = bf16_rne(fl32(c[q] * s_hat))."""
+    q = unpack(codes)
+    n, k = q.shape
+    s_hat = restored_scale_code(q2, gdata, code)
+    c = codebook()
+    prod = (c[q].reshape(-1, BLOCK) * s_hat.reshape(-1, 1)).astype(np.float32)
+    return round_f32_to_bf16_bits(prod).reshape(n, k)
+
+
+def dequantize_code(codes, q2, gdata, code):
+    return bf16_bits_to_f32(dequantize_bits_code(codes, q2, gdata, code))
+
+
+def storage_bytes_code(n, k, code):
+    """Bytes of the stored format with scale code `code`: (codes, scale codes, group data)."""
+    nb = n * k // BLOCK
+    return n * k // 2, nb, 4 * group_data_floats(code) * n_groups(nb)
+
+
+def bits_per_param_code(n, k, code):
+    return 8.0 * sum(storage_bytes_code(n, k, code)) / float(n * k)

@@ -77,3 +77,33 @@ def test_single_rank_helpers_are_identity():
     t = torch.ones(3)
     bench.allreduce_grads([t], 1)
     assert torch.equal(t, torch.ones(3))
+
+
+def test_bench_launcher_starts_n_ranks(tmp_path):
+    # bench.py --gpus N outside a launcher re-runs itself as N ranks under
+    # torch.distributed.run; here the same launcher starts a small script
+    # that joins a gloo group and reports its rank and the world size
+    import json
+    import subprocess
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    script = tmp_path / "rank_report.py"
+    out = tmp_path / "ranks"
+    out.mkdir()
+    script.write_text(
+        "import os, json, torch.distributed as dist\n"
+        "from datetime import timedelta\n"
+        "dist.init_process_group('gloo', timeout=timedelta(seconds=60))\n"
+        "r, w = dist.get_rank(), dist.get_world_size()\n"
+        "dist.barrier()\n"
+        f"open(os.path.join({str(out)!r}, f'r{{r}}.json'), 'w').write(json.dumps(dict(rank=r, world=w, "
+        "local=int(os.environ['LOCAL_RANK']))))\n"
+        "dist.destroy_process_group()\n")
+    cmd = bench.torchrun_command(2, str(script), [], bench.free_port())
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"] and "--nproc-per-node=2" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    rc = bench.spawn_ranks(2, str(script), [], timeout_s=240)
+    assert rc == 0
+    got = sorted((json.loads((out / f"r{i}.json").read_text()) for i in range(2)), key=lambda d: d["rank"])
+    assert [(d["rank"], d["world"], d["local"]) for d in got] == [(0, 2, 0), (1, 2, 1)]

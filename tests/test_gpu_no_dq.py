@@ -56,7 +56,8 @@ def test_gemm_restore_exact_without_dq(q):
 
 
 @pytest.mark.parametrize("n,k,m,r,path", [(512, 512, 300, 8, "gemm"), (384, 1024, 16, 64, "gemm"),
-                                          (4096, 4096, 1, 64, "gemv"), (1000, 512, 9, 12, "gemv")])
+                                          (4096, 4096, 1, 64, "gemv"), (1000, 512, 9, 12, "gemv"),
+                                          (1000, 192, 5, 8, "gemv"), (24, 4096, 1, 16, "gemv")])
 def test_forward_parity_without_dq(q, n, k, m, r, path):
     alpha = 16.0
     w = synth.weight(n, k, seed=k + m, outliers=True)

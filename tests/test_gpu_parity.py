@@ -215,6 +215,10 @@ FWD_CASES = [
     (4096, 4096, 1, 64, "gemv"),     # decode shape
     (1000, 512, 3, 12, "gemv"),
     (1000, 512, 9, 12, "gemv"),      # two token groups
+    (1001, 192, 1, 8, "gemv"),       # 3 blocks per row, ragged last row group
+    (37, 64, 16, 8, "gemv"),         # one block per row, 16 tokens
+    (8, 11008, 2, 64, "gemv"),       # eight rows, a long reduction
+    (22016, 256, 1, 16, "gemv"),     # many row groups, short rows
 ]
 
 
@@ -279,24 +283,30 @@ def test_forward_narrow_tiles_parity(q, n, k, m, r):
     assert linear.rel_fro(_np(u), (alpha / r) * u_ref) <= TOL
 
 
-def test_forward_gemv_restores_w_exactly(q):
-    n, k, r = 256, 512, 8
-    w = synth.weight(n, k, seed=6)
+@pytest.mark.parametrize("n,k", [(256, 512), (1001, 4096), (64, 192)])
+def test_forward_gemv_restores_w_exactly(q, n, k):
+    # one-hot tokens pick out columns of W_hat: the decode GEMV restores each
+    # weight exactly as the standalone restore does, so y equals those
+    # columns bit for bit (d_out 1001: a ragged last row group; d_in 192:
+    # three blocks per row)
+    r = 8
+    w = synth.weight(n, k, seed=6, outliers=True)
     o = _oracle_quant(w)
     qw = q.qlora_quantize_nf4(w.cuda())
     ref = nf4.dequantize_bits(o["codes"], o["q2"], o["smax"])
     b = torch.zeros((n, r), dtype=torch.bfloat16)
     a = synth.lora_a(r, k)
-    for k0 in (0, 77, 511):
-        x = torch.zeros((3, k), dtype=torch.bfloat16)
-        x[0, k0] = 1
-        x[2, (k0 + 5) % k] = 1
-        y, _ = q.qlora_linear_fwd_ex(qw, x.cuda(), a.cuda(), b.cuda(), 16.0, path=q.FWD_GEMV)
-        torch.cuda.synchronize()
-        yb = _bits(y)
-        assert np.array_equal(yb[0], ref[:, k0])
-        assert np.array_equal(yb[2], ref[:, (k0 + 5) % k])
-        assert np.all(yb[1] == 0)
+    for k0 in (0, 77, k - 1):
+        for m in (3, 12):
+            x = torch.zeros((m, k), dtype=torch.bfloat16)
+            x[0, k0] = 1
+            x[2, (k0 + 5) % k] = 1
+            y, _ = q.qlora_linear_fwd_ex(qw, x.cuda(), a.cuda(), b.cuda(), 16.0, path=q.FWD_GEMV)
+            torch.cuda.synchronize()
+            yb = _bits(y)
+            assert np.array_equal(yb[0], ref[:, k0])
+            assert np.array_equal(yb[2], ref[:, (k0 + 5) % k])
+            assert np.all(yb[1] == 0)
 
 
 def test_forward_w_zero_is_lora_only(q):

@@ -473,3 +473,110 @@ def test_no_dq_restore_matches_brute_force_and_bound():
     # error within half the largest level gap of the block scale, plus bf16 rounding
     s_b = np.repeat(o["absmax"].reshape(6, 2), 64, axis=1)
     assert np.all(np.abs(w - got) <= s_b * nf4.max_level_gap() / 2 + np.abs(got) * 2.0 ** -8 + 1e-30)
+
+
+# --------------------------------------------------------------------------- scale-code variants
+# The 255-step unsigned grid and the signed mid-range code, both readings of
+# the same double-quantization paragraph (8-bit codes of the block scales,
+# 32-bit constants per group, error bounded by the grid step).
+
+def _scales(n, seed, spread=1.0):
+    g = np.random.default_rng(seed)
+    s = np.abs(g.normal(0.05, 0.01 * spread, size=n)).astype(np.float32)
+    return bf16.round_to_bf16(s)
+
+
+@pytest.mark.parametrize("code", ["u8_255", "s8_mid"])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_scale_codes_match_brute_force(code, seed):
+    # 600 scales: two full groups and a short one, with a zero scale, a
+    # repeated maximum and an outlier
+    s = _scales(600, seed)
+    s[5] = 0.0
+    s[300] = s[301] = np.float32(0.5)
+    s[599] = np.float32(3.0)
+    q2, gd = nf4.double_quantize_code(s, code)
+    sh = nf4.restored_scale_code(q2, gd, code)
+    if code == "u8_255":
+        q_b, smax_b, sh_b = brute.double_quantize_u8_255([float(v) for v in s])
+        assert np.array_equal(q2.astype(np.int64), np.array(q_b))
+        assert np.array_equal(gd, np.array(smax_b, np.float32))
+    else:
+        q_b, gd_b, sh_b = brute.double_quantize_s8_mid([float(v) for v in s])
+        assert np.array_equal(q2.view(np.int8).astype(np.int64), np.array(q_b))
+        assert np.array_equal(gd, np.array(gd_b, np.float32))
+    assert np.array_equal(sh.view(np.uint32), np.array(sh_b, np.float32).view(np.uint32))
+
+
+def test_scale_code_u8_255_bound_and_top_code():
+    # |s - s_hat| <= s_max / 510 up to float32 rounding (the float32 ratio can
+    # move a code on a half-step by up to 255 * 2^-23 of a step, and the
+    # restore rounds once more: a slack of 2^-20 s_max covers both); the
+    # group maximum is exact
+    s = _scales(256 * 8, 3, spread=3.0)
+    q2, smax = nf4.double_quantize_code(s, "u8_255")
+    sh = nf4.restored_scale_code(q2, smax, "u8_255")
+    g = np.arange(s.size) // 256
+    err = np.abs(s.astype(np.float64) - sh.astype(np.float64))
+    assert np.all(err <= smax[g].astype(np.float64) * (1.0 / 510.0 + 2.0 ** -20))
+    top = s == smax[g]
+    assert np.all(q2[top] == 255) and np.array_equal(sh[top], s[top])
+    # and it is never worse than the printed 1/256 grid's bound
+    assert err.max() <= smax.max() / 256.0
+
+
+def test_scale_code_s8_mid_bound_and_centering():
+    # |s - s_hat| <= half / 254 up to float32 rounding (half = half the
+    # group's spread); the centred code beats the printed grid on N(0, 0.02)
+    # weights, whose block scales sit close together
+    w = _w(512, 1024, seed=4)
+    a = nf4.block_absmax(w)
+    q2, gd = nf4.double_quantize_code(a, "s8_mid")
+    sh = nf4.restored_scale_code(q2, gd, "s8_mid")
+    g = np.arange(a.size) // 256
+    half = gd[g, 1].astype(np.float64)
+    err = np.abs(a.astype(np.float64) - sh.astype(np.float64))
+    assert np.all(err <= half / 254.0 + 2.0 ** -22 * np.abs(a))
+    q2u, smax = nf4.double_quantize(a)
+    err_u = np.abs(a.astype(np.float64) - nf4.restored_scale(q2u, smax).astype(np.float64))
+    # the signed step 2 half / 254 against the printed s_max / 256: with the
+    # mean half / s_max of these groups (about 0.3) the error ratio is about 0.6
+    ratio = 2.0 * 256.0 / 254.0 * float(np.mean(gd[:, 1] / nf4.group_smax(a)))
+    assert np.sqrt(np.mean(err ** 2)) < min(0.75, 1.15 * ratio) * np.sqrt(np.mean(err_u ** 2))
+    assert q2.view(np.int8).min() == -127 and q2.view(np.int8).max() == 127
+
+
+def test_scale_code_special_groups():
+    # a group of equal scales (half = 0: every code 0, s_hat = s exactly), an
+    # all-zero group, and the 255-grid's zero group
+    s = np.concatenate([np.full(256, 0.0625, np.float32), np.zeros(256, np.float32)])
+    q2, gd = nf4.double_quantize_code(s, "s8_mid")
+    assert np.all(q2 == 0) and np.array_equal(nf4.restored_scale_code(q2, gd, "s8_mid"), s)
+    q2, smax = nf4.double_quantize_code(s, "u8_255")
+    assert np.all(q2[256:] == 0) and np.all(q2[:256] == 255)
+    assert np.array_equal(nf4.restored_scale_code(q2, smax, "u8_255"), s)
+
+
+def test_scale_code_bit_budgets():
+    # 4-bit codes + an 8-bit scale code per 64 weights + the group constants
+    # per 256 blocks (16384 weights): one float32 for the unsigned codes, two
+    # for the signed one
+    n, k = 1024, 4096
+    assert nf4.bits_per_param_code(n, k, "u8_255") == pytest.approx(4 + 8 / 64 + 32 / 16384, abs=0)
+    assert nf4.bits_per_param_code(n, k, "u8_256") == nf4.bits_per_param(n, k)
+    assert nf4.bits_per_param_code(n, k, "s8_mid") == pytest.approx(4 + 8 / 64 + 64 / 16384, abs=0)
+    assert round(nf4.bits_per_param_code(n, k, "u8_255"), 2) == _golden("bit_budget.json")["bits_nf4_double_quant"]
+
+
+@pytest.mark.parametrize("code", ["u8_255", "s8_mid"])
+def test_restore_with_scale_code_is_bf16_of_level_times_scale(code):
+    w = _w(8, 640, seed=7, outliers=True)
+    o = nf4.quantize_code(w, code)
+    bits = nf4.dequantize_bits_code(o["codes"], o["q2"], o["gdata"], code)
+    sh = nf4.restored_scale_code(o["q2"], o["gdata"], code)
+    c = [float(v) for v in nf4.codebook()]
+    for i in range(0, 8 * 640, 97):
+        r, kk = divmod(i, 640)
+        q = int(o["q"][r, kk])
+        want = brute.bf16_round_bits(brute.Fraction(brute.f32_round(brute.Fraction(c[q]) * brute.Fraction(float(sh[i // 64])))))
+        assert int(bits[r, kk]) == want
