@@ -20,7 +20,7 @@ import os
 
 __all__ = [
     "LIB_PATH", "lib", "QloraError", "NF4Weight", "Nf4Struct",
-    "qlora_nf4_bytes", "qlora_nf4_codebook", "qlora_quantize_nf4", "qlora_dequantize",
+    "qlora_nf4_bytes", "qlora_nf4_codebook", "DQ_U8_256", "DQ_U8_255", "DQ_S8_MID", "qlora_quantize_nf4", "qlora_dequantize",
     "qlora_workspace_bytes", "qlora_fwd_workspace_bytes", "qlora_linear_fwd", "qlora_linear_fwd_ex", "qlora_linear_fwd_noalloc",
     "qlora_linear_bwd",
     "qlora_device_status", "qlora_status_string", "qlora_version", "qlora_launch_count",
@@ -54,6 +54,8 @@ class Nf4Struct(ctypes.Structure):
         ("codes", ctypes.c_void_p),
         ("scale_codes", ctypes.c_void_p),
         ("absmax", ctypes.c_void_p),
+        ("dq_code", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
     ]
 
 
@@ -61,6 +63,8 @@ _vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ct
 _P = ctypes.POINTER
 lib.qlora_nf4_bytes.argtypes = [_i64, _i64, _i32, _P(_sz)]
 lib.qlora_nf4_bytes.restype = _sz
+lib.qlora_nf4_bytes_ex.argtypes = [_i64, _i64, _i32, _i32, _P(_sz)]
+lib.qlora_nf4_bytes_ex.restype = _sz
 lib.qlora_nf4_codebook.argtypes = [_P(ctypes.c_float)]
 lib.qlora_nf4_codebook.restype = ctypes.c_int
 lib.qlora_quantize_nf4.argtypes = [_vp, _P(Nf4Struct), _vp]
@@ -161,10 +165,14 @@ def qlora_status_string(status):
     return lib.qlora_status_string(int(status)).decode()
 
 
-def qlora_nf4_bytes(n_out, k_in, dq_group=256):
+# scale codes of the double quantization (qlora_dq_code_t)
+DQ_U8_256, DQ_U8_255, DQ_S8_MID = 0, 1, 2
+
+
+def qlora_nf4_bytes(n_out, k_in, dq_group=256, dq_code=DQ_U8_256):
     """(codes, scale codes, group constants) byte sizes of the stored format."""
     out = (ctypes.c_size_t * 3)()
-    total = lib.qlora_nf4_bytes(int(n_out), int(k_in), int(dq_group), out)
+    total = lib.qlora_nf4_bytes_ex(int(n_out), int(k_in), int(dq_group), int(dq_code), out)
     if total == 0:
         raise QloraError(2, "qlora_nf4_bytes")
     return int(out[0]), int(out[1]), int(out[2])
@@ -179,13 +187,15 @@ def qlora_nf4_codebook():
 
 class NF4Weight:
     """Device buffers of one packed NF4 weight. dq=True: codes, 8-bit scale
-    codes and one s_max per 256 blocks (double quantization); dq=False:
-    codes and one fp32 scale per 64-weight block (no scale codes)."""
+    codes and the group constants of `dq_code` per 256 blocks (double
+    quantization); dq=False: codes and one fp32 scale per 64-weight block (no
+    scale codes)."""
 
-    def __init__(self, n_out, k_in, device="cuda", dq=True):
+    def __init__(self, n_out, k_in, device="cuda", dq=True, dq_code=DQ_U8_256):
         torch = _torch()
         self.dq = bool(dq)
-        b_codes, b_q2, b_smax = qlora_nf4_bytes(n_out, k_in, 256 if self.dq else 0)
+        self.dq_code = int(dq_code) if self.dq else DQ_U8_256
+        b_codes, b_q2, b_smax = qlora_nf4_bytes(n_out, k_in, 256 if self.dq else 0, self.dq_code)
         self.n_out, self.k_in = int(n_out), int(k_in)
         self.codes = torch.empty(b_codes, dtype=torch.uint8, device=device)
         self.scale_codes = torch.empty(b_q2, dtype=torch.uint8, device=device)
@@ -194,17 +204,18 @@ class NF4Weight:
     def struct(self):
         q2 = self.scale_codes.data_ptr() if self.dq else 0
         return Nf4Struct(self.n_out, self.k_in, 64, 256 if self.dq else 0, self.codes.data_ptr(), q2,
-                         self.absmax.data_ptr())
+                         self.absmax.data_ptr(), self.dq_code, 0)
 
     def nbytes(self):
         return self.codes.numel() + self.scale_codes.numel() + 4 * self.absmax.numel()
 
 
-def qlora_quantize_nf4(w, out=None, stream=None, dq=True):
+def qlora_quantize_nf4(w, out=None, stream=None, dq=True, dq_code=DQ_U8_256):
     """Quantize a bf16 CUDA weight [N, K] into an :class:`NF4Weight` (with
-    double quantization unless dq=False or `out` says otherwise)."""
+    double quantization in scale code `dq_code` unless dq=False, or as `out`
+    says)."""
     assert w.is_cuda and w.dim() == 2 and w.is_contiguous()
-    q = out if out is not None else NF4Weight(w.shape[0], w.shape[1], device=w.device, dq=dq)
+    q = out if out is not None else NF4Weight(w.shape[0], w.shape[1], device=w.device, dq=dq, dq_code=dq_code)
     s = q.struct()
     _check(lib.qlora_quantize_nf4(_ptr(w), ctypes.byref(s), _stream_ptr(stream)), "qlora_quantize_nf4")
     return q

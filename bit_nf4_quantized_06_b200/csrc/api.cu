@@ -369,6 +369,9 @@ qlora_status_t check_nf4(const qlora_nf4_t* q) {
   if (q == nullptr || q->codes == nullptr || q->absmax == nullptr) return QLORA_ERR_INVALID_ARG;
   if (q->block != kBlock || (q->dq_group != kGroup && q->dq_group != 0)) return QLORA_ERR_INVALID_ARG;
   if (q->dq_group == kGroup && q->scale_codes == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (q->dq_group == kGroup && (q->dq_code < QLORA_DQ_U8_256 || q->dq_code > QLORA_DQ_S8_MID))
+    return QLORA_ERR_INVALID_ARG;
+  if (q->reserved != 0) return QLORA_ERR_INVALID_ARG;
   if (q->n_out <= 0 || q->k_in <= 0 || q->k_in % kBlock != 0) return QLORA_ERR_SHAPE;
   if (q->n_out > (int64_t(1) << 31) - 1 || q->k_in > (int64_t(1) << 31) - 1) return QLORA_ERR_SHAPE;
   if (!aligned16(q->codes)) return QLORA_ERR_ALIGNMENT;
@@ -465,7 +468,9 @@ qlora_status_t launch_pair(int pairs, int64_t m, cudaStream_t st, const CUtensor
       return QLORA_ERR_CUDA;
     p.tma_out = 1;
   }
-  p.tiles_cols = static_cast<int32_t>(cdiv(m, 256 * pair_nh(m)));
+  // the signed scale code's two group constants need the NH = 1 restore slots
+  const int nh = (p.dq && p.dqc == QLORA_DQ_S8_MID) ? 1 : pair_nh(m);
+  p.tiles_cols = static_cast<int32_t>(cdiv(m, 256 * nh));
   p.feat_n = 256;
   p.tiles_rows = static_cast<int32_t>(cdiv(p.rows, 256));
   const int64_t tiles = static_cast<int64_t>(p.tiles_rows) * p.tiles_cols;
@@ -486,7 +491,7 @@ qlora_status_t launch_pair(int pairs, int64_t m, cudaStream_t st, const CUtensor
     p.feat_n = pick_feat_n(p.rows, p.tiles_cols, pairs);
     p.tiles_rows = static_cast<int32_t>(cdiv(p.rows, p.feat_n));
   }
-  if (pair_nh(m) == 2) return launch_pair_nh<AS, 2>(pairs, st, b, bl, c, o, p);
+  if (nh == 2) return launch_pair_nh<AS, 2>(pairs, st, b, bl, c, o, p);
   return launch_pair_nh<AS, 1>(pairs, st, b, bl, c, o, p);
 }
 
@@ -564,7 +569,7 @@ using namespace qlora;
 
 extern "C" {
 
-int32_t qlora_version(void) { return 100; }
+int32_t qlora_version(void) { return 10100; }
 
 uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -597,19 +602,25 @@ qlora_status_t qlora_nf4_codebook(float out[16]) {
   return QLORA_OK;
 }
 
-size_t qlora_nf4_bytes(int64_t n_out, int64_t k_in, int32_t dq_group, size_t out[3]) {
+size_t qlora_nf4_bytes_ex(int64_t n_out, int64_t k_in, int32_t dq_group, int32_t dq_code, size_t out[3]) {
   if (n_out <= 0 || k_in <= 0 || k_in % kBlock != 0 || (dq_group != kGroup && dq_group != 0)) return 0;
+  if (dq_group == kGroup && (dq_code < QLORA_DQ_U8_256 || dq_code > QLORA_DQ_S8_MID)) return 0;
   const int64_t nb = n_out * k_in / kBlock;
   const bool dq = dq_group == kGroup;
   const size_t b0 = static_cast<size_t>(n_out * k_in / 2);
   const size_t b1 = dq ? static_cast<size_t>(nb) : 0;
-  const size_t b2 = static_cast<size_t>(dq ? cdiv(nb, kGroup) : nb) * sizeof(float);
+  const int64_t per_group = (dq && dq_code == QLORA_DQ_S8_MID) ? 2 : 1;   // group constants
+  const size_t b2 = static_cast<size_t>(dq ? per_group * cdiv(nb, kGroup) : nb) * sizeof(float);
   if (out) {
     out[0] = b0;
     out[1] = b1;
     out[2] = b2;
   }
   return b0 + b1 + b2;
+}
+
+size_t qlora_nf4_bytes(int64_t n_out, int64_t k_in, int32_t dq_group, size_t out[3]) {
+  return qlora_nf4_bytes_ex(n_out, k_in, dq_group, QLORA_DQ_U8_256, out);
 }
 
 namespace {
@@ -647,6 +658,7 @@ qlora_status_t qlora_quantize_nf4(const void* w_bf16, const qlora_nf4_t* q, void
   std::memcpy(qp.cell_m, tables().cell_m, sizeof(qp.cell_m));
   std::memcpy(qp.cell_below, tables().cell_below, sizeof(qp.cell_below));
   qp.dq = q->dq_group == kGroup ? 1 : 0;
+  qp.dqc = qp.dq ? q->dq_code : 0;
   const int64_t groups = cdiv(nb, kGroup);
   if (groups > 0x7FFFFFFF) return QLORA_ERR_SHAPE;
   k_quantize_nf4<<<static_cast<unsigned>(groups), 256, 0, static_cast<cudaStream_t>(stream)>>>(
@@ -666,6 +678,7 @@ qlora_status_t qlora_dequantize(const qlora_nf4_t* q, void* w_bf16_out, void* st
   DequantParams dp{};
   std::memcpy(dp.cb, tables().cb, sizeof(dp.cb));
   dp.dq = q->dq_group == kGroup ? 1 : 0;
+  dp.dqc = dp.dq ? q->dq_code : 0;
   const int blocks = static_cast<int>(std::min<int64_t>(cdiv(nwords, 256), int64_t(sms) * 16));
   k_dequantize_nf4<<<std::max(blocks, 1), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const uint32_t*>(q->codes), q->scale_codes, q->absmax, nwords,
@@ -759,6 +772,7 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
     gp.ldb = static_cast<int32_t>(ldb);
     std::memcpy(gp.cb, tables().cb, sizeof(gp.cb));
     gp.dq = q->dq_group == kGroup ? 1 : 0;
+    gp.dqc = gp.dq ? q->dq_code : 0;
     // launched as a programmatic dependent of the x A^T kernel: its weight
     // stream starts while u' is still being computed
     cudaLaunchConfig_t cfg = {};
@@ -804,6 +818,7 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
   p.kblocks = k / 64;
   p.nblocks = n * (k / 64);
   p.dq = q->dq_group == kGroup ? 1 : 0;
+  p.dqc = p.dq ? q->dq_code : 0;
   p.w_rows = n;
   p.w_cols = k;
   std::memcpy(p.cb, tables().cb, sizeof(p.cb));
@@ -929,6 +944,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
     p.kblocks = k / 64;
     p.nblocks = n * (k / 64);
     p.dq = q->dq_group == kGroup ? 1 : 0;
+    p.dqc = p.dq ? q->dq_code : 0;
     p.w_rows = n;
     p.w_cols = k;
     std::memcpy(p.cb, tables().cb, sizeof(p.cb));
@@ -987,6 +1003,7 @@ qlora_status_t qlora_merge_lora(const qlora_nf4_t* q, const void* a, const void*
   p.s = alpha / static_cast<float>(r);
   std::memcpy(p.cb, tables().cb, sizeof(p.cb));
   p.dq = q->dq_group == kGroup ? 1 : 0;
+  p.dqc = p.dq ? q->dq_code : 0;
   const size_t smem = merge_smem_bytes(p.r64);
   const dim3 grid(static_cast<unsigned>(cdiv(p.k, 128)), static_cast<unsigned>(cdiv(p.n, 128)), 1);
   if (grid.y > 65535u) return QLORA_ERR_SHAPE;

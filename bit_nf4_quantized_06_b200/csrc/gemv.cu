@@ -102,37 +102,38 @@ __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
   struct Chunk {
     uint4 a_lo, a_hi, b_lo, b_hi;
     uint32_t q2a, q2b;
-    float sma, smb;
+    float sma, smb, sma2, smb2;   // group constants (the second only for the signed scale code)
+  };
+  // the group constants of block bi (dq) or its fp32 scale (no dq)
+  auto scale_data = [&](int64_t bi, uint32_t& q2, float& c0, float& c1) {
+    if (!p.dq) {
+      c0 = __ldg(p.smax + bi);          // fp32 block scale, no double quantization
+    } else if (p.dqc == 2) {
+      q2 = __ldg(p.q2 + bi);
+      c0 = __ldg(p.smax + 2 * (bi >> 8));
+      c1 = __ldg(p.smax + 2 * (bi >> 8) + 1);
+    } else {
+      q2 = __ldg(p.q2 + bi);
+      c0 = __ldg(p.smax + (bi >> 8));
+    }
   };
   auto fetch = [&](int64_t c, Chunk& ch) {
     const int64_t kb = c * 4 + qd;
     const bool kv = c < nchunks && kb < kpr;
     ch.a_lo = ch.a_hi = ch.b_lo = ch.b_hi = make_uint4(0, 0, 0, 0);
     ch.q2a = ch.q2b = 0;
-    ch.sma = ch.smb = 0.0f;
+    ch.sma = ch.smb = ch.sma2 = ch.smb2 = 0.0f;
     if (kv && v0) {
       const uint8_t* src = p.codes + r0 * row_bytes + kb * 32;
       ch.a_lo = ldg_stream(src);
       ch.a_hi = ldg_stream(src + 16);
-      const int64_t bi = r0 * kpr + kb;
-      if (p.dq) {
-        ch.q2a = __ldg(p.q2 + bi);
-        ch.sma = __ldg(p.smax + (bi >> 8));
-      } else {
-        ch.sma = __ldg(p.smax + bi);     // fp32 block scale, no double quantization
-      }
+      scale_data(r0 * kpr + kb, ch.q2a, ch.sma, ch.sma2);
     }
     if (kv && v1) {
       const uint8_t* src = p.codes + r1 * row_bytes + kb * 32;
       ch.b_lo = ldg_stream(src);
       ch.b_hi = ldg_stream(src + 16);
-      const int64_t bi = r1 * kpr + kb;
-      if (p.dq) {
-        ch.q2b = __ldg(p.q2 + bi);
-        ch.smb = __ldg(p.smax + (bi >> 8));
-      } else {
-        ch.smb = __ldg(p.smax + bi);     // fp32 block scale, no double quantization
-      }
+      scale_data(r1 * kpr + kb, ch.q2b, ch.smb, ch.smb2);
     }
   };
 
@@ -146,8 +147,8 @@ __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
   for (int64_t c = warp; c < nchunks; c += WARPS) {
     const int64_t kb = c * 4 + qd;
     const bool kv = kb < kpr;
-    const Nf4Table t0 = make_table(p.cb, p.dq ? restored_scale(cur.q2a, cur.sma) : cur.sma);
-    const Nf4Table t1 = make_table(p.cb, p.dq ? restored_scale(cur.q2b, cur.smb) : cur.smb);
+    const Nf4Table t0 = make_table(p.cb, p.dq ? dq_block_scale(cur.q2a, cur.sma, cur.sma2, p.dqc) : cur.sma);
+    const Nf4Table t1 = make_table(p.cb, p.dq ? dq_block_scale(cur.q2b, cur.smb, cur.smb2, p.dqc) : cur.smb);
     const uint32_t wa[8] = {cur.a_lo.x, cur.a_lo.y, cur.a_lo.z, cur.a_lo.w,
                             cur.a_hi.x, cur.a_hi.y, cur.a_hi.z, cur.a_hi.w};
     const uint32_t wb[8] = {cur.b_lo.x, cur.b_lo.y, cur.b_lo.z, cur.b_lo.w,

@@ -13,7 +13,8 @@ namespace qlora {
 extern __device__ unsigned int g_dev_status;
 
 struct QuantParams {
-  int32_t dq;     // 1: q2 codes + group s_max; 0: fp32 block scale into absmax
+  int32_t dq;     // 1: q2 codes + group constants; 0: fp32 block scale into absmax
+  int32_t dqc;    // scale code (qlora_dq_code_t) when dq
   // cut[j] (j < 15): the real number halfway between m_j (the fp32 midpoint
   // of levels j and j+1) and the next float32 above m_j; a quotient rounds
   // to a float32 above m_j exactly when it exceeds cut[j]. cut[15] is padding.
@@ -33,7 +34,8 @@ constexpr float kEncodeGuard = 5e-7f;
 
 struct DequantParams {
   float cb[16];   // the 16 fp32 levels
-  int32_t dq;     // 1: s_hat from q2 and s_max; 0: absmax holds s_b per block
+  int32_t dq;     // 1: s_hat from q2 and the group constants; 0: absmax holds s_b per block
+  int32_t dqc;    // scale code (qlora_dq_code_t) when dq: 2 has two constants per group
 };
 
 __global__ void k_quantize_nf4(const uint4* __restrict__ w, int64_t nb, uint32_t* __restrict__ codes,
@@ -54,7 +56,8 @@ struct GemvParams {
   __nv_bfloat16* y;       // [M x N]
   int64_t n, k;
   int32_t m, r, r64, ldb;
-  int32_t dq;             // 1: s_hat from q2 and s_max; 0: smax holds s_b per block
+  int32_t dq;             // 1: s_hat from q2 and the group constants; 0: smax holds s_b per block
+  int32_t dqc;            // scale code (qlora_dq_code_t) when dq: 2 has two constants per group
   float cb[16];
 };
 
@@ -95,7 +98,9 @@ struct TcParams {
   const float* smax;
   int64_t kblocks;      // K/64 of the weight: blocks per weight row
   int64_t nblocks;      // N*K/64: length of q2
-  int32_t dq;           // 1: s_hat from q2 and s_max; 0: smax holds s_b per block
+  int32_t dq;           // 1: s_hat from q2 and the group constants; 0: smax holds s_b per block
+  int32_t dqc;          // scale code (qlora_dq_code_t) when dq: 2 has two constants per group
+                        // (only with NH = 1: its restore slots have room for both)
   int64_t w_rows;       // N of the weight (rows of W)
   int64_t w_cols;       // K of the weight
   float cb[16];
@@ -174,9 +179,14 @@ __global__ void k_tc_pair(const __grid_constant__ CUtensorMap tm_b, const __grid
                           const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_out,
                           TcParams p);
 
+// bytes of scale data per restore thread and k-tile in the pair kernels: the
+// q2 word and one group constant (8), or with room for the signed scale
+// code's second constant (16; NH = 1 only, NH = 2 has no shared memory left)
+constexpr uint32_t pair_scale_slot(int nh) { return nh == 1 ? 16u : 8u; }
+
 constexpr int tc_pair_smem_bytes(int nh) {
-  return pair_stages(nh) * (16384 + nh * 16384 + 4096) + 1024 + 256 + 2 * kScalePrefetch * 128 * 8 +
-         kPairEpiStage;
+  return pair_stages(nh) * (16384 + nh * 16384 + 4096) + 1024 + 256 +
+         2 * kScalePrefetch * 128 * static_cast<int>(pair_scale_slot(nh)) + kPairEpiStage;
 }
 
 __global__ void k_reduce_splits(SmallParams p);
@@ -194,7 +204,8 @@ struct MergeParams {
   int64_t n, k;
   int32_t r, r64;
   float s;
-  int32_t dq;               // 1: s_hat from q2 and s_max; 0: smax holds s_b per block
+  int32_t dq;               // 1: s_hat from q2 and the group constants; 0: smax holds s_b per block
+  int32_t dqc;              // scale code (qlora_dq_code_t) when dq: 2 has two constants per group
   float cb[16];
 };
 __global__ void k_merge_lora(MergeParams p);

@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(256, 2) k_merge_lora(MergeParams p) {
   const int64_t kpr = p.k >> 6;
   uint32_t cw[8];
   uint32_t cq2[8];
-  float csm[8];
+  float csm[8], csm2[8];    // group constants (the second only for the signed scale code)
 #pragma unroll
   for (int it = 0; it < 8; ++it) {
     const int c = tid + 256 * it;
@@ -85,16 +85,20 @@ __global__ void __launch_bounds__(256, 2) k_merge_lora(MergeParams p) {
     const int64_t n = n0 + row, kc = k0 + c8 * 8;
     cw[it] = 0;
     cq2[it] = 0;
-    csm[it] = 0.0f;
+    csm[it] = csm2[it] = 0.0f;
     if (n < p.n && kc < p.k) {
       const int64_t e0 = n * p.k + kc;
       cw[it] = __ldcs(reinterpret_cast<const uint32_t*>(p.codes) + (e0 >> 3));
       const int64_t blk = n * kpr + (kc >> 6);
-      if (p.dq) {
+      if (!p.dq) {
+        csm[it] = __ldg(p.smax + blk);     // fp32 block scale, no double quantization
+      } else if (p.dqc == 2) {
+        cq2[it] = __ldg(p.q2 + blk);
+        csm[it] = __ldg(p.smax + 2 * (blk >> 8));
+        csm2[it] = __ldg(p.smax + 2 * (blk >> 8) + 1);
+      } else {
         cq2[it] = __ldg(p.q2 + blk);
         csm[it] = __ldg(p.smax + (blk >> 8));
-      } else {
-        csm[it] = __ldg(p.smax + blk);     // fp32 block scale, no double quantization
       }
     }
   }
@@ -210,7 +214,7 @@ __global__ void __launch_bounds__(256, 2) k_merge_lora(MergeParams p) {
     if (n >= p.n || kc >= p.k) continue;
     const int64_t e0 = n * p.k + kc;                 // first element of the chunk
     const uint32_t w = cw[it];
-    const float sh = p.dq ? restored_scale(cq2[it], csm[it]) : csm[it];
+    const float sh = p.dq ? dq_block_scale(cq2[it], csm[it], csm2[it], p.dqc) : csm[it];
     const float4 dlo = *reinterpret_cast<const float4*>(sD + row * LDD + c8 * 8);
     const float4 dhi = *reinterpret_cast<const float4*>(sD + row * LDD + c8 * 8 + 4);
     const float d[8] = {dlo.x, dlo.y, dlo.z, dlo.w, dhi.x, dhi.y, dhi.z, dhi.w};

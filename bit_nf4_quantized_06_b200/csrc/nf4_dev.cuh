@@ -33,6 +33,17 @@ __device__ __forceinline__ float restored_scale(uint32_t q2, float smax) {
   return __fmul_rn(prod, 0.00390625f);  // 2^-8, exact except for subnormal results
 }
 
+// Block scale of a scale code (qlora_dq_code_t; the formulas of the ABI
+// header): c0 = s_max (or mid), c1 = half (signed code only).
+__device__ __forceinline__ float dq_block_scale(uint32_t q2, float c0, float c1, int code) {
+  if (code == 1) return __fdiv_rn(__fmul_rn(static_cast<float>(q2), c0), 255.0f);
+  if (code == 2) {
+    const float q = static_cast<float>(static_cast<int>(static_cast<int8_t>(static_cast<uint8_t>(q2))));
+    return __fadd_rn(c0, __fdiv_rn(__fmul_rn(q, c1), 127.0f));
+  }
+  return restored_scale(q2, c0);
+}
+
 // cb: the 16 fp32 levels (kernel-parameter constants).
 __device__ __forceinline__ Nf4Table make_table(const float (&cb)[16], float s_hat) {
   uint32_t p[8];

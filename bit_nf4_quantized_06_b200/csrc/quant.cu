@@ -11,6 +11,9 @@
 //   byte  = (q[2i] << 4) | q[2i+1]
 //   s_max = max s_b over 256 consecutive blocks (the last group may be short)
 //   q2    = min(255, rint_even(fl32(256 * s_b / s_max)))   (0 if s_max == 0)
+// or one of the two further scale codes (qlora_dq_code_t in the ABI header:
+// the 255-step grid, or the signed code centred on the group's mid-range,
+// which also needs the group's minimum scale).
 //
 // One CTA of 256 threads owns one double-quantization group (256 blocks,
 // 16384 weights, 32 KB of bf16): every thread loads 8 x 16 B with fully
@@ -107,6 +110,7 @@ __global__ void __launch_bounds__(256, 3) k_quantize_nf4(const uint4* __restrict
   __shared__ float s_tab[66];     // [0, 33): the midpoint in each cell; [33, 66): midpoints below it
   __shared__ double s_cut[16];
   __shared__ uint32_t s_wmax[8];
+  __shared__ uint32_t s_wmin[8];
   const int tid = threadIdx.x;
   const int64_t g = blockIdx.x;
   const int64_t b0 = g * 256;
@@ -126,7 +130,7 @@ __global__ void __launch_bounds__(256, 3) k_quantize_nf4(const uint4* __restrict
   if (tid < 16) s_cut[tid] = qp.cut[tid];
 
   uint32_t am[8];
-  uint32_t gm = 0;
+  uint32_t gm = 0, gn = 0xFFFFu;   // group max, and min over the group's blocks (not its padding)
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     uint32_t m = abs_bits_max(v[i]);
@@ -135,14 +139,23 @@ __global__ void __launch_bounds__(256, 3) k_quantize_nf4(const uint4* __restrict
     m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
     am[i] = m;
     gm = max(gm, m);
+    gn = min(gn, ((tid >> 3) + 32 * i < nblk) ? m : 0xFFFFu);
   }
   gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 8));
   gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 16));
-  if ((tid & 31) == 0) s_wmax[tid >> 5] = gm;
+  gn = min(gn, __shfl_xor_sync(0xFFFFFFFFu, gn, 8));
+  gn = min(gn, __shfl_xor_sync(0xFFFFFFFFu, gn, 16));
+  if ((tid & 31) == 0) {
+    s_wmax[tid >> 5] = gm;
+    s_wmin[tid >> 5] = gn;
+  }
   __syncthreads();
-  uint32_t gmax = s_wmax[0];
+  uint32_t gmax = s_wmax[0], gmin = s_wmin[0];
 #pragma unroll
-  for (int i = 1; i < 8; ++i) gmax = max(gmax, s_wmax[i]);
+  for (int i = 1; i < 8; ++i) {
+    gmax = max(gmax, s_wmax[i]);
+    gmin = min(gmin, s_wmin[i]);
+  }
   const float s_max = __uint_as_float(gmax << 16);
   // per-block outputs: the eight lanes of a block group each take one of
   // the group's eight blocks, (tid >> 3) + 32 * (tid & 7)
@@ -154,12 +167,33 @@ __global__ void __launch_bounds__(256, 3) k_quantize_nf4(const uint4* __restrict
   if (!qp.dq) {
     // 4.5-bit format: the block scale itself is stored (exact: a bf16 magnitude)
     if (my_bi < nblk) smax[b0 + my_bi] = __uint_as_float(my_am << 16);
+  } else if (qp.dqc == 2) {
+    // signed code centred on the group's mid-range: two constants per group
+    const float lo = __uint_as_float(gmin << 16);
+    const float mid = __fmul_rn(__fadd_rn(lo, s_max), 0.5f);
+    const float half = __fmul_rn(__fsub_rn(s_max, lo), 0.5f);
+    if (tid == 0) {
+      smax[2 * g] = mid;
+      smax[2 * g + 1] = half;
+    }
+    if (my_bi < nblk) {
+      int code = 0;
+      if (half != 0.0f) {
+        const float t = __fsub_rn(__uint_as_float(my_am << 16), mid);
+        const float ratio = __fdiv_rn(__fmul_rn(127.0f, t), half);
+        code = max(-127, min(127, __float2int_rn(ratio)));
+      }
+      q2[b0 + my_bi] = static_cast<uint8_t>(static_cast<int8_t>(code));
+    }
   } else {
     if (tid == 0) smax[g] = s_max;
     if (my_bi < nblk) {
       uint32_t code = 0;
       if (s_max != 0.0f) {
-        const float ratio = __fdiv_rn(256.0f * __uint_as_float(my_am << 16), s_max);
+        // 256 steps (the printed grid; 256 s is exact) or 255 steps
+        const float num = qp.dqc == 1 ? __fmul_rn(255.0f, __uint_as_float(my_am << 16))
+                                      : 256.0f * __uint_as_float(my_am << 16);
+        const float ratio = __fdiv_rn(num, s_max);
         code = static_cast<uint32_t>(min(255, __float2int_rn(ratio)));
       }
       q2[b0 + my_bi] = static_cast<uint8_t>(code);
@@ -250,7 +284,14 @@ __global__ void __launch_bounds__(256) k_dequantize_nf4(const uint32_t* __restri
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nwords;
        i += stride) {
     const int64_t b = i >> 3;
-    const float s_hat = dp.dq ? restored_scale(__ldg(q2 + b), __ldg(smax + (b >> 8))) : __ldg(smax + b);
+    float s_hat;
+    if (!dp.dq) {
+      s_hat = __ldg(smax + b);
+    } else if (dp.dqc == 2) {
+      s_hat = dq_block_scale(__ldg(q2 + b), __ldg(smax + 2 * (b >> 8)), __ldg(smax + 2 * (b >> 8) + 1), 2);
+    } else {
+      s_hat = dq_block_scale(__ldg(q2 + b), __ldg(smax + (b >> 8)), 0.0f, dp.dqc);
+    }
     const uint32_t w = __ldcs(codes + i);
     uint32_t o[4];
 #pragma unroll

@@ -237,7 +237,10 @@ __global__ void __launch_bounds__(448, 1)
     const int grp = (warp - 2) >> 2;                 // 0: warps 2-5, 1: warps 6-9
     const int tid = threadIdx.x - 64 - 128 * grp;    // 0..127
     const int items = work.items;
-    const uint32_t slot0 = ring + grp * (PD * 128 * 8) + tid * 8;
+    // scale slot per thread and k-tile: the q2 word and the group constant(s)
+    // (the signed scale code's two constants need the 16-byte slot of NH = 1)
+    constexpr uint32_t SLOT = pair_scale_slot(NH);
+    const uint32_t slot0 = ring + grp * (PD * 128 * SLOT) + tid * SLOT;
 
     // cursor over this group's items j = grp, grp + 2, ... of the pair's
     // work list: k-tile t (< k1) of segment i, whose restored slice starts at
@@ -274,12 +277,17 @@ __global__ void __launch_bounds__(448, 1)
     auto issue = [&](const Cursor& c, int k) {
       if (c.j < items && c.t < p.kt_main) {
         const int64_t bi = block_of(c.f0, c.t);
-        const uint32_t slot = slot0 + k * (128 * 8);
+        const uint32_t slot = slot0 + k * (128 * SLOT);
         if (bi >= 0 && p.dq) {
           const int64_t w4 = bi & ~int64_t(3);
           const int64_t left = p.nblocks - w4;
           cp_async4(slot, p.q2 + w4, static_cast<uint32_t>(left < 4 ? left : 4));
-          cp_async4(slot + 4, p.smax + (bi >> 8), 4);
+          if (SLOT == 16 && p.dqc == 2) {
+            cp_async4(slot + 4, p.smax + 2 * (bi >> 8), 4);
+            cp_async4(slot + 8, p.smax + 2 * (bi >> 8) + 1, 4);
+          } else {
+            cp_async4(slot + 4, p.smax + (bi >> 8), 4);
+          }
         } else if (bi >= 0) {
           cp_async4(slot, p.smax, 0);
           cp_async4(slot + 4, p.smax + bi, 4);     // fp32 block scale, no double quantization
@@ -323,13 +331,14 @@ __global__ void __launch_bounds__(448, 1)
       if (t < p.kt_main) {
         cp_async_wait<PD - 1>();
         const int64_t bi = block_of(f0, t);
-        const uint32_t slot = slot0 + slot_use * (128 * 8);
+        const uint32_t slot = slot0 + slot_use * (128 * SLOT);
         float sh = 0.0f;
         if (bi >= 0) {
           if (p.dq) {
             const uint32_t qw = lds32(slot);
             const uint32_t q2 = (qw >> (8 * static_cast<uint32_t>(bi & 3))) & 0xFFu;
-            sh = restored_scale(q2, __uint_as_float(lds32(slot + 4)));
+            const float c1 = (SLOT == 16 && p.dqc == 2) ? __uint_as_float(lds32(slot + 8)) : 0.0f;
+            sh = dq_block_scale(q2, __uint_as_float(lds32(slot + 4)), c1, p.dqc);
           } else {
             sh = __uint_as_float(lds32(slot + 4));
           }

@@ -78,15 +78,36 @@ typedef enum {
   QLORA_ERR_TIMEOUT = 7            /* a kernel gave up on a bounded wait            */
 } qlora_status_t;
 
+/* Code of the 8-bit block-scale code under double quantization (the
+ * 8-bit scale codes with 32-bit constants per group of 256 scales of
+ * «QLoRA는 어떻게 65B 모델을 GPU 한 장에 올렸나», § "메모리 회계: 세 겹의
+ * 최적화"; the sources print the first, the other two are readings of the
+ * same paragraph). Per group of 256 consecutive block scales s:
+ *   QLORA_DQ_U8_256: one fp32 constant s_max = max s;
+ *     q2 = min(255, rint(fl32(fl32(256 s) / s_max))) (unsigned),
+ *     s_hat = fl32(q2 * s_max) * 2^-8; error at most s_max / 256.
+ *   QLORA_DQ_U8_255: one fp32 constant s_max;
+ *     q2 = min(255, rint(fl32(fl32(255 s) / s_max))) (unsigned),
+ *     s_hat = fl32(fl32(q2 * s_max) / 255); error at most s_max / 510.
+ *   QLORA_DQ_S8_MID: two fp32 constants mid = fl32(fl32(lo + hi) / 2) and
+ *     half = fl32(fl32(hi - lo) / 2) (lo, hi = min, max s), stored as
+ *     [mid, half] per group; q2 = clamp(rint(fl32(fl32(127 fl32(s - mid)) /
+ *     half)), -127, 127) stored as an int8 byte (0 when half is 0),
+ *     s_hat = fl32(mid + fl32(fl32(q2 * half) / 127)); error at most
+ *     half / 254. rint rounds half to even. */
+typedef enum { QLORA_DQ_U8_256 = 0, QLORA_DQ_U8_255 = 1, QLORA_DQ_S8_MID = 2 } qlora_dq_code_t;
+
 /* Packed NF4 weight. All pointers are device pointers owned by the caller;
- * sizes from qlora_nf4_bytes(). Two formats («QLoRA는 어떻게 65B 모델을 GPU 한
+ * sizes from qlora_nf4_bytes_ex(). Formats («QLoRA는 어떻게 65B 모델을 GPU 한
  * 장에 올렸나», § "메모리 회계: 세 겹의 최적화"):
  *   dq_group = 256: double quantization (~4.13 bits/param): scale_codes holds
- *     one 8-bit code q2 per 64-weight block and absmax one fp32 s_max per 256
- *     consecutive blocks; the block scale is s_hat = fl32(q2 * s_max) * 2^-8;
+ *     one 8-bit code q2 per 64-weight block, absmax the group constants of
+ *     dq_code (one float per 256 consecutive blocks, or two for
+ *     QLORA_DQ_S8_MID); with QLORA_DQ_U8_256 the block scale is
+ *     s_hat = fl32(q2 * s_max) * 2^-8;
  *   dq_group = 0: no double quantization (4.5 bits/param): absmax holds the
  *     fp32 block scale s_b itself, one per block; scale_codes is unused and
- *     may be NULL. */
+ *     may be NULL; dq_code is ignored. */
 typedef struct {
   int64_t n_out;         /* N rows (d_out)                                     */
   int64_t k_in;          /* K columns (d_in), K % 64 == 0                      */
@@ -94,17 +115,24 @@ typedef struct {
   int32_t dq_group;      /* 256 (double quantization) or 0 (none)              */
   uint8_t *codes;        /* N*K/2 bytes                                        */
   uint8_t *scale_codes;  /* N*K/64 bytes (dq_group 256), unused for 0          */
-  float *absmax;         /* ceil(N*K/64/256) s_max (dq_group 256), or N*K/64
-                            block scales (dq_group 0)                          */
+  float *absmax;         /* group constants (dq_group 256: 1 or 2 floats per
+                            ceil(N*K/64/256) groups), or N*K/64 block scales
+                            (dq_group 0); 4-byte aligned                       */
+  int32_t dq_code;       /* qlora_dq_code_t (dq_group 256)                     */
+  int32_t reserved;      /* must be 0                                          */
 } qlora_nf4_t;
 
 /* Forward path selection for qlora_linear_fwd_ex. AUTO takes the decode GEMV
  * for m <= 16 and the tensor-core GEMM otherwise. */
 typedef enum { QLORA_FWD_AUTO = 0, QLORA_FWD_GEMM = 1, QLORA_FWD_GEMV = 2 } qlora_fwd_path_t;
 
-/* Byte sizes of the three stored arrays (codes, scale codes, fp32 scales)
- * for dq_group 256 or 0; returns their sum (0 on bad shape or dq_group).
- * out may be NULL. Host only, no device work. */
+/* Byte sizes of the three stored arrays (codes, scale codes, fp32 scales or
+ * group constants) for dq_group 256 or 0 and scale code dq_code; returns
+ * their sum (0 on bad shape, dq_group or dq_code). out may be NULL. Host
+ * only, no device work. */
+QLORA_API size_t qlora_nf4_bytes_ex(int64_t n_out, int64_t k_in, int32_t dq_group, int32_t dq_code, size_t out[3]);
+
+/* qlora_nf4_bytes_ex with dq_code QLORA_DQ_U8_256. */
 QLORA_API size_t qlora_nf4_bytes(int64_t n_out, int64_t k_in, int32_t dq_group, size_t out[3]);
 
 /* The library's own fp32 NF4 table (16 ascending levels in [-1, 1] with an
@@ -314,7 +342,8 @@ QLORA_API const char *qlora_status_string(qlora_status_t s);
  * device work behind a sequence of calls. */
 QLORA_API uint64_t qlora_launch_count(void);
 
-/* Library version as major*10000 + minor*100 + patch. */
+/* Library version as major*10000 + minor*100 + patch (1.1.0: qlora_nf4_t
+ * gained dq_code and reserved). */
 QLORA_API int32_t qlora_version(void);
 
 #ifdef __cplusplus

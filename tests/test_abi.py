@@ -145,3 +145,21 @@ def test_gemm_schedule_setting(q):
             assert q.qlora_fwd_workspace_bytes(4096, 4096, 4096, 64) < forced
     finally:
         q.qlora_set_gemm_schedule(q.SCHED_AUTO)
+
+
+def test_nf4_bytes_of_the_scale_codes(q):
+    # the unsigned codes keep one float32 per group of 256 block scales, the
+    # signed mid-range code two; the scale codes themselves are one byte each
+    n, k = 4096, 4096
+    nb, ng = n * k // 64, (n * k // 64 + 255) // 256
+    assert q.qlora_nf4_bytes(n, k, 256, q.DQ_U8_256) == (n * k // 2, nb, 4 * ng)
+    assert q.qlora_nf4_bytes(n, k, 256, q.DQ_U8_255) == (n * k // 2, nb, 4 * ng)
+    assert q.qlora_nf4_bytes(n, k, 256, q.DQ_S8_MID) == (n * k // 2, nb, 8 * ng)
+    assert q.lib.qlora_nf4_bytes_ex(n, k, 256, 3, None) == 0          # unknown code
+    assert q.lib.qlora_nf4_bytes_ex(n, k, 0, 7, None) > 0             # ignored without DQ
+    # rejected before any device work: unknown code, nonzero reserved field
+    s = q.Nf4Struct(512, 512, 64, 256, 16, 16, 16, 3, 0)
+    assert q.lib.qlora_dequantize(ctypes.byref(s), ctypes.c_void_p(16), None) == 1
+    s = q.Nf4Struct(512, 512, 64, 256, 16, 16, 16, 0, 1)
+    assert q.lib.qlora_dequantize(ctypes.byref(s), ctypes.c_void_p(16), None) == 1
+    assert q.qlora_version() == 10100
