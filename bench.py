@@ -607,6 +607,82 @@ def cpu_baseline_sample(target_s=15.0):
     }
 
 
+def oracle_config_timings():
+    """The oracle (as it stands) timed on the host cores for every workload,
+    each on a bounded sample (a few seconds each), in the unit of its GPU
+    figure: the tiny problem in full; the decode call (restore of the full
+    4096x4096 weight, then the fp64 forward of one token); the 65B gate/up
+    projection's quantizer on 1024 of its 22016 rows and its fp64 fwd+bwd on
+    16 tokens over those rows; the whole stack's quantizer on 512 rows of
+    each of its seven projection shapes."""
+    from oracle import linear, nf4
+    cores = len(os.sched_getaffinity(0))
+    out = {"cores": cores, "kind": "oracle"}
+
+    def f64(t):
+        return t.float().numpy().astype(np.float64)
+
+    def quantize_restore(w):
+        o = nf4.quantize(w)
+        return nf4.dequantize(o["codes"], o["q2"], o["smax"]).astype(np.float64)
+
+    # tiny: quantize + fwd + bwd in full, repeated for about a second
+    p = synth.TINY
+    t = synth.make(p)
+    w, x, a, b, dy = t["w"].float().numpy(), f64(t["x"]), f64(t["a"]), f64(t["b"]), f64(t["dy"])
+    reps, t0 = 0, time.perf_counter()
+    while reps < 3 or time.perf_counter() - t0 < 1.0:
+        wh = quantize_restore(w)
+        linear.forward(x, wh, a, b, p.scale)
+        linear.backward(x, dy, wh, a, b, p.scale)
+        reps += 1
+    dt = (time.perf_counter() - t0) / reps
+    out["tiny"] = {"workload": p.name, "us_per_step": round(dt * 1e6, 1),
+                   "TFLOP/s": round((fwd_flops(p.m, p.n, p.k, p.r) + bwd_flops(p.m, p.n, p.k, p.r)) / dt / 1e12, 6),
+                   "sample": "full problem: quantize, restore, fp64 forward and backward"}
+    # decode: restore the whole weight, then one token's forward (the GEMV's bytes per call)
+    p = synth.DECODE
+    t = synth.make(p)
+    t0 = time.perf_counter()
+    wh = quantize_restore(t["w"].float().numpy())
+    t1 = time.perf_counter()
+    linear.forward(f64(t["x"]), wh, f64(t["a"]), f64(t["b"]), p.scale)
+    t2 = time.perf_counter()
+    out["decode"] = {"workload": p.name, "ms_per_call": round((t2 - t1) * 1e3, 3),
+                     "GB/s": round(gemv_bytes(p.n, p.k, p.r) / (t2 - t1) / 1e9, 3),
+                     "quantize_restore_s": round(t1 - t0, 3),
+                     "sample": "full weight restored once (not timed per call); fp64 forward of one token"}
+    # 65B gate/up: quantizer and fwd+bwd on a row sample
+    p = synth.GATE65B
+    rows = 1024
+    w = synth.weight(rows, p.k, seed=0, outliers=True).float().numpy()
+    t0 = time.perf_counter()
+    wh = quantize_restore(w)
+    tq = time.perf_counter() - t0
+    tok = 16
+    x, a, b, dy = (f64(synth.tokens(tok, p.k)), f64(synth.lora_a(p.r, p.k)), f64(synth.lora_b(rows, p.r)),
+                   f64(synth.grad_out(tok, rows)))
+    t0 = time.perf_counter()
+    linear.forward(x, wh, a, b, p.scale)
+    linear.backward(x, dy, wh, a, b, p.scale)
+    tl = time.perf_counter() - t0
+    out["65b_gate_up"] = {"workload": p.name, "quantize_GB/s": round(quant_bytes(rows, p.k) / tq / 1e9, 4),
+                          "fwd_bwd_TFLOP/s": round((fwd_flops(tok, rows, p.k, p.r) + bwd_flops(tok, rows, p.k, p.r))
+                                                   / tl / 1e12, 4),
+                          "sample": f"{rows} of {p.n} rows quantized and restored; fp64 fwd+bwd of {tok} tokens over those rows"}
+    # whole stack: the quantizer on 512 rows of each projection shape
+    rows, qb, tq = 512, 0, 0.0
+    for idx, (_, n, k) in enumerate(synth.STACK7B_LAYER):
+        w = synth.weight(rows, k, seed=idx).float().numpy()
+        t0 = time.perf_counter()
+        quantize_restore(w)
+        tq += time.perf_counter() - t0
+        qb += quant_bytes(rows, k)
+    out["stack_quantize"] = {"workload": "whole 7B-shaped stack quantizer", "GB/s": round(qb / tq / 1e9, 4),
+                             "sample": f"{rows} rows of each of the seven projection shapes (of 6,476,005,376 weights)"}
+    return out
+
+
 def run_ours(args):
     world, rank, local = dist_env()
     if world > 1:
@@ -752,6 +828,7 @@ def run_ours(args):
         line["whole_stack"] = stack
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_sample()
+        line["cpu_baseline_configs"] = oracle_config_timings()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
