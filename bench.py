@@ -251,10 +251,12 @@ def flush_l2(buf):
     buf.add_(1)
 
 
-def gemv_steady_state(q, device, calls=200, copies=32):
+DECODE65 = synth.Problem("decode-gemv-22016x8192-m1-r64", 22016, 8192, 1, 64, 16.0, backward=False)
+
+
+def gemv_steady_state(q, device, calls=200, copies=32, d=synth.DECODE):
     """Decode GEMV per call in steady state: a CUDA graph of `calls` back-to-back
     forwards cycling over `copies` packed weights (> 2x L2)."""
-    d = synth.DECODE
     t = synth.make(d, seed=77)
     x, a, b = t["x"].to(device), t["a"].to(device), t["b"].to(device)
     w0 = q.qlora_quantize_nf4(t["w"].to(device))
@@ -560,12 +562,115 @@ def whole_stack(q, device, l2):
         raise RuntimeError(f"device status {st} ({bits:#x}) in the stack sweep")
     fl = sum(fwd_flops(m, n, k, r) + bwd_flops(m, n, k, r) for _, n, k, _, _ in lin)
     qb = sum(quant_bytes(n, k) for _, n, k, _, _ in lin)
+    popt = stack_paged_optimizer(q, lin, xs, dys, ys, dxs, ws, m, r, alpha, l2)
     del lin
-    return {"weights": params, "linears": 224, "quantize_ms": round(q_ms, 3),
+    return {"weights": params, "linears": 224, "quantize_ms": round(q_ms, 3), "paged_optimizer": popt,
             "quantize_GB/s": round(qb / (q_ms * 1e-3) / 1e9, 1), "fwd_bwd_ms": round(t_ms, 3),
             "fwd_bwd_TFLOP": round(fl / 1e12, 2), "fwd_bwd_TFLOP/s": round(fl / (t_ms * 1e-3) / 1e12, 1),
             "workload": "whole 7B-shaped stack, 32 x (q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008), "
                         "4096 tokens, r=64, weights generated on the GPU per layer"}
+
+
+def stack_paged_optimizer(q, lin, xs, dys, ys, dxs, ws, m, r, alpha, l2, steps=3):
+    """The optimizer's cost per training step of the whole stack, the unit in
+    which the pages quote the paged optimizer's throughput loss. One step is
+    the forward of all 224 quantized linears (each saving its u'), then their
+    backward in reverse order; as soon as a linear's dA, dB are written, the
+    AdamW update of its adapter pair (160,067,584 parameters over the stack)
+    is queued on a second stream, so the updates overlap the rest of the
+    backward, and the step ends when both streams are done. The update runs
+    four ways: none; the GPU kernel with m, v in device memory; the GPU
+    kernel with m, v paged out to pinned host memory (read and written over
+    the host link); the CPU update (gradient copied to the host, AdamW on the
+    host cores, bf16 adapter copied back). Medians of `steps` steps, L2
+    flushed before each."""
+    dev = xs[4096].device
+    sizes = [r * k + n * r for _, n, k, _, _ in lin]
+    offs = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+    total = int(offs[-1])
+    param = torch.empty(total, dtype=torch.bfloat16, device=dev)
+    grad = torch.zeros(total, dtype=torch.float32, device=dev)
+    views = []
+    for i, (qw, n, k, a, b) in enumerate(lin):
+        o = int(offs[i])
+        pa, pb = param[o:o + r * k].view(r, k), param[o + r * k:o + sizes[i]].view(n, r)
+        pa.copy_(a)
+        pb.copy_(b)
+        views.append((pa, pb, grad[o:o + r * k].view(r, k), grad[o + r * k:o + sizes[i]].view(n, r)))
+    master = param.float()
+    m_d, v_d = torch.zeros(total, device=dev), torch.zeros(total, device=dev)
+    m_h, v_h = torch.zeros(total).pin_memory(), torch.zeros(total).pin_memory()
+    master_h = param.float().cpu().pin_memory()
+    grad_h = torch.empty(total).pin_memory()
+    param_h = torch.empty(total, dtype=torch.bfloat16).pin_memory()
+    us = [torch.empty((m, r), dtype=torch.bfloat16, device=dev) for _ in lin]
+    side = torch.cuda.Stream(device=dev)
+    hp = dict(lr=1e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0)
+    evs = [torch.cuda.Event() for _ in lin]
+
+    def update_fn(kind):
+        def dev_states(i, t):
+            o, e = int(offs[i]), int(offs[i + 1])
+            q.qlora_adamw_step(master[o:e], grad[o:e], m_d[o:e], v_d[o:e], t, param=param[o:e], stream=side, **hp)
+
+        def host_states(i, t):
+            o, e = int(offs[i]), int(offs[i + 1])
+            q.qlora_adamw_step(master[o:e], grad[o:e], m_h[o:e], v_h[o:e], t, param=param[o:e], stream=side, **hp)
+
+        def cpu(i, t):
+            o, e = int(offs[i]), int(offs[i + 1])
+            q.qlora_adamw_paged(grad[o:e], master_h[o:e], m_h[o:e], v_h[o:e], grad_h[o:e], t, param_dev=param[o:e],
+                                param_host=param_h[o:e], stream=side, **hp)
+        return {"none": None, "gpu_device_states": dev_states, "gpu_host_states": host_states,
+                "cpu_paged": cpu}[kind]
+
+    def step(upd, t):
+        main = torch.cuda.current_stream()
+        for i, (qw, n, k, a, b) in enumerate(lin):
+            pa, pb, _, _ = views[i]
+            q.qlora_linear_fwd(qw, xs[k], pa, pb, alpha, y=ys[n], u=us[i], ws=ws)
+        for i in reversed(range(len(lin))):
+            qw, n, k, _, _ = lin[i]
+            pa, pb, ga, gb = views[i]
+            q.qlora_linear_bwd(qw, xs[k], us[i], dys[n], pa, pb, alpha, dx=dxs[k], da=ga, db=gb, ws=ws)
+            if upd is not None:
+                evs[i].record(main)
+                side.wait_event(evs[i])
+                upd(i, t)
+        if upd is not None:
+            main.wait_stream(side)
+
+    out, t = {}, 0
+    for kind in ("none", "gpu_device_states", "gpu_host_states", "cpu_paged"):
+        upd = update_fn(kind)
+        t += 1
+        step(upd, t)                        # warm-up
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(steps):
+            t += 1
+            flush_l2(l2)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            step(upd, t)
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        out[kind] = float(np.median(times))
+    st, bits = q.qlora_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({bits:#x}) in the stack training steps")
+    base = out["none"]
+    res = {"adapter_params": total, "step_ms_no_update": round(base, 3),
+           "method": "224 forwards then 224 backwards in reverse; each pair's AdamW queued on a second stream "
+                     "when its dA, dB are written; medians of %d steps" % steps}
+    for kind in ("gpu_device_states", "gpu_host_states", "cpu_paged"):
+        res[kind] = {"step_ms": round(out[kind], 3), "throughput_loss": round(out[kind] / base - 1.0, 4)}
+    res["gpu_host_states"]["host_link_bytes_per_step"] = 16 * total
+    res["cpu_paged"]["cpu_threads"] = os.cpu_count()
+    res["pages_quote"] = "about 8% throughput loss for the paged optimizer"
+    return res
 
 
 def cpu_baseline_sample(target_s=15.0):
@@ -752,6 +857,8 @@ def run_ours(args):
         gemv_ms, gemv_lat_ms, _ = gemv_steady_state(q, device)
         gb = gemv_bytes(d.n, d.k, d.r)
         gemv_gbs = gb / (gemv_ms * 1e-3) / 1e9
+        g65_ms, g65_lat_ms, _ = gemv_steady_state(q, device, calls=50, copies=4, d=DECODE65)
+        g65_b = gemv_bytes(DECODE65.n, DECODE65.k, DECODE65.r)
 
     # end to end through host buffers: H2D of x, dY, W; D2H of dA, dB and the decode output
     e2e_ms = None
@@ -817,7 +924,13 @@ def run_ours(args):
                         "us_single_call": round(gemv_lat_ms * 1e3, 3), "bytes_per_call": gb,
                         "GB/s": round(gemv_gbs, 1), "frac_hbm": round(gemv_gbs / peaks["hbm_gbs"], 4),
                         "peak_hbm_gbs": peaks["hbm_gbs"], "frac_vs_8tbs": round(gemv_gbs / 8000.0, 4),
-                        "method": "CUDA graph of 200 calls over 32 rotating packed weights (277 MB > 2x L2), x5 replays"}
+                        "method": "CUDA graph of 200 calls over 32 rotating packed weights (277 MB > 2x L2), x5 replays",
+                        "65b_gate": {"workload": DECODE65.name, "us_per_call_steady": round(g65_ms * 1e3, 3),
+                                     "us_single_call": round(g65_lat_ms * 1e3, 3), "bytes_per_call": g65_b,
+                                     "GB/s": round(g65_b / (g65_ms * 1e-3) / 1e9, 1),
+                                     "frac_hbm": round(g65_b / (g65_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                                     "method": "CUDA graph of 50 calls over 4 rotating packed weights "
+                                               "(367 MB > 2x L2), x5 replays"}}
         line["merge"] = {"workload": p.name + " LoRA merge for export, bf16(W_hat + s B A)", "ms": round(merge_ms, 4),
                          "bytes": int(mb), "GB/s": round(mb / (merge_ms * 1e-3) / 1e9, 1),
                          "frac_hbm": round(mb / (merge_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
