@@ -515,25 +515,30 @@ def gemm_schedule(q, device, l2, reps=5):
 def whole_stack(q, device, l2):
     """The whole 7B-shaped stack: 32 layers of q, k, v, o (4096x4096), gate,
     up (11008x4096) and down (4096x11008), 6,476,005,376 weights ~ N(0, 0.02).
-    Each weight is generated on the GPU from its own seed, quantized (NF4 +
-    double quantization; CUDA events around the quantize calls only) and its
-    bf16 copy freed. Then forward + backward of all 224 quantized linears at
-    4096 tokens with r = 64 adapters, one event pair around the whole sweep."""
+    Each weight is generated on the GPU from its own seed; the 224 quantize
+    calls (NF4 + double quantization) then run back to back inside one event
+    pair, and the bf16 copies are freed. Then forward + backward of all 224
+    quantized linears at 4096 tokens with r = 64 adapters, one event pair
+    around the whole sweep."""
     m, r, alpha = 4096, 64, 16.0
-    lin, params, q_ms = [], 0, 0.0
+    lin, ws_bf16, params = [], [], 0
     for layer in range(synth.STACK7B_LAYERS):
         for idx, (_, n, k) in enumerate(synth.STACK7B_LAYER):
             w, a, b = synth.stack_linear(layer, idx, r=r, device=device)
-            qw = q.NF4Weight(n, k, device=device)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            q.qlora_quantize_nf4(w, out=qw)
-            e1.record()
-            torch.cuda.synchronize()
-            q_ms += e0.elapsed_time(e1)
-            del w
-            lin.append((qw, n, k, a, b))
+            ws_bf16.append(w)
+            lin.append((q.NF4Weight(n, k, device=device), n, k, a, b))
             params += n * k
+    # all 224 quantize calls back to back (12.95 GB of bf16 in, resident)
+    flush_l2(l2)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for w, (qw, _, _, _, _) in zip(ws_bf16, lin):
+        q.qlora_quantize_nf4(w, out=qw)
+    e1.record()
+    torch.cuda.synchronize()
+    q_ms = e0.elapsed_time(e1)
+    del ws_bf16
     xs, dys = synth.stack_activations(m, device=device)
     ys = {n: torch.empty((m, n), dtype=torch.bfloat16, device=device) for n in (4096, 11008)}
     dxs = {k: torch.empty((m, k), dtype=torch.bfloat16, device=device) for k in (4096, 11008)}

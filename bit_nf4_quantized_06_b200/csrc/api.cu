@@ -12,6 +12,7 @@
 
 #include "../../include/qlora.h"
 #include "kernels.h"
+#include "nf4_dev.cuh"
 #include "ptx.cuh"
 
 namespace qlora {
@@ -221,6 +222,9 @@ qlora_status_t device_ready(int* sms_out, int* pairs_out = nullptr) {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_merge_lora, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(merge_smem_bytes(kMaxRank)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_merge_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(merge_tc_smem_bytes()));
     if (e != cudaSuccess) return QLORA_ERR_CUDA;
     st.attrs = true;
     st.ctx = ctx;
@@ -782,7 +786,12 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = (m <= 8) ? cudaLaunchKernelEx(&cfg, k_gemv_nf4<1>, gp) : cudaLaunchKernelEx(&cfg, k_gemv_nf4<2>, gp);
+    // one instantiation per token-group count and block-scale format
+    using GemvKernel = void (*)(GemvParams);
+    static constexpr GemvKernel kGemv[2][4] = {
+        {k_gemv_nf4<1, kScNone>, k_gemv_nf4<1, kScU8x256>, k_gemv_nf4<1, kScU8x255>, k_gemv_nf4<1, kScS8Mid>},
+        {k_gemv_nf4<2, kScNone>, k_gemv_nf4<2, kScU8x256>, k_gemv_nf4<2, kScU8x255>, k_gemv_nf4<2, kScS8Mid>}};
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kGemv[m <= 8 ? 0 : 1][scale_format(gp.dq, gp.dqc)], gp);
     if (e != cudaSuccess) {
       g_launches.fetch_add(1, std::memory_order_relaxed);
       cudaGetLastError();
@@ -1004,10 +1013,27 @@ qlora_status_t qlora_merge_lora(const qlora_nf4_t* q, const void* a, const void*
   std::memcpy(p.cb, tables().cb, sizeof(p.cb));
   p.dq = q->dq_group == kGroup ? 1 : 0;
   p.dqc = p.dq ? q->dq_code : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the tensor-core merge takes B through TMA (16-byte rows: r % 8 == 0)
+  if (r % 8 == 0) {
+    CUtensorMap m_b, m_a, m_codes, m_out;
+    if (!map_bf16(&m_b, b, p.n, r, r, 128) || !map_bf16(&m_a, a, r, p.k, p.k, 64) ||
+        !map2d(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->codes, static_cast<uint64_t>(p.k / 2),
+               static_cast<uint64_t>(p.n), static_cast<uint64_t>(p.k / 2), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map2d(&m_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_out, static_cast<uint64_t>(p.k), static_cast<uint64_t>(p.n),
+               static_cast<uint64_t>(p.k) * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+      return QLORA_ERR_CUDA;
+    p.tiles_n = static_cast<int32_t>(cdiv(p.n, 128));
+    p.tiles_k = static_cast<int32_t>(cdiv(p.k, 256));
+    const int64_t tiles = static_cast<int64_t>(p.tiles_n) * p.tiles_k;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, sms));
+    k_merge_tc<<<grid, 32 * (2 + kMergeDrainWarps), merge_tc_smem_bytes(), st>>>(m_b, m_a, m_codes, m_out, p);
+    return launch_status();
+  }
   const size_t smem = merge_smem_bytes(p.r64);
   const dim3 grid(static_cast<unsigned>(cdiv(p.k, 128)), static_cast<unsigned>(cdiv(p.n, 128)), 1);
   if (grid.y > 65535u) return QLORA_ERR_SHAPE;
-  k_merge_lora<<<grid, 256, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  k_merge_lora<<<grid, 256, smem, st>>>(p);
   return launch_status();
 }
 

@@ -59,7 +59,7 @@ __device__ __forceinline__ uint32_t ld_bf16_pair(const __nv_bfloat16* row, int j
 
 }  // namespace
 
-template <int NT>
+template <int NT, int SC>
 __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
   constexpr int WARPS = 8;
   __shared__ float s_red[WARPS][32][NT * 4];
@@ -106,9 +106,9 @@ __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
   };
   // the group constants of block bi (dq) or its fp32 scale (no dq)
   auto scale_data = [&](int64_t bi, uint32_t& q2, float& c0, float& c1) {
-    if (!p.dq) {
+    if constexpr (SC == kScNone) {
       c0 = __ldg(p.smax + bi);          // fp32 block scale, no double quantization
-    } else if (p.dqc == 2) {
+    } else if constexpr (SC == kScS8Mid) {
       q2 = __ldg(p.q2 + bi);
       c0 = __ldg(p.smax + 2 * (bi >> 8));
       c1 = __ldg(p.smax + 2 * (bi >> 8) + 1);
@@ -147,8 +147,8 @@ __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
   for (int64_t c = warp; c < nchunks; c += WARPS) {
     const int64_t kb = c * 4 + qd;
     const bool kv = kb < kpr;
-    const Nf4Table t0 = make_table(p.cb, p.dq ? dq_block_scale(cur.q2a, cur.sma, cur.sma2, p.dqc) : cur.sma);
-    const Nf4Table t1 = make_table(p.cb, p.dq ? dq_block_scale(cur.q2b, cur.smb, cur.smb2, p.dqc) : cur.smb);
+    const Nf4Table t0 = make_table(p.cb, block_scale_sc<SC>(cur.q2a, cur.sma, cur.sma2));
+    const Nf4Table t1 = make_table(p.cb, block_scale_sc<SC>(cur.q2b, cur.smb, cur.smb2));
     const uint32_t wa[8] = {cur.a_lo.x, cur.a_lo.y, cur.a_lo.z, cur.a_lo.w,
                             cur.a_hi.x, cur.a_hi.y, cur.a_hi.z, cur.a_hi.w};
     const uint32_t wb[8] = {cur.b_lo.x, cur.b_lo.y, cur.b_lo.z, cur.b_lo.w,
@@ -225,8 +225,14 @@ __global__ void __launch_bounds__(256, 2) k_gemv_nf4(GemvParams p) {
   }
 }
 
-template __global__ void k_gemv_nf4<1>(GemvParams);
-template __global__ void k_gemv_nf4<2>(GemvParams);
+template __global__ void k_gemv_nf4<1, kScNone>(GemvParams);
+template __global__ void k_gemv_nf4<1, kScU8x256>(GemvParams);
+template __global__ void k_gemv_nf4<1, kScU8x255>(GemvParams);
+template __global__ void k_gemv_nf4<1, kScS8Mid>(GemvParams);
+template __global__ void k_gemv_nf4<2, kScNone>(GemvParams);
+template __global__ void k_gemv_nf4<2, kScU8x256>(GemvParams);
+template __global__ void k_gemv_nf4<2, kScU8x255>(GemvParams);
+template __global__ void k_gemv_nf4<2, kScS8Mid>(GemvParams);
 
 // u'[m][j] = bf16(s * sum_k x[m][k] A[j][k]) for M <= 16 (the decode LoRA
 // down projection). Rank j is owned by four warps (one per quarter of K)

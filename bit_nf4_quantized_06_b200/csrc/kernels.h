@@ -73,7 +73,8 @@ struct LoraDownSmallParams {
   float s;
 };
 
-template <int NT>
+// NT token groups of 8; SC the block-scale format (kScNone .. kScS8Mid of nf4_dev.cuh)
+template <int NT, int SC>
 __global__ void k_gemv_nf4(GemvParams p);
 template <int MT>
 __global__ void k_lora_down_small(LoraDownSmallParams p);
@@ -207,8 +208,24 @@ struct MergeParams {
   int32_t dq;               // 1: s_hat from q2 and the group constants; 0: smax holds s_b per block
   int32_t dqc;              // scale code (qlora_dq_code_t) when dq: 2 has two constants per group
   float cb[16];
+  int32_t tiles_n, tiles_k; // tensor-core merge: 128-row x 256-column output tiles
 };
 __global__ void k_merge_lora(MergeParams p);
+
+// Tensor-core merge (B rows 16-byte aligned, r % 8 == 0): persistent CTAs,
+// s B A for a 128 x 256 tile in tensor memory (tcgen05, operands by TMA), the
+// restore, add and rounding in the drain, output by TMA stores.
+//   tm_b: B [N x r] bf16, boxes {64, 128}; tm_a: A [r x K] bf16, boxes {64, 64};
+//   tm_codes: codes [N x K/2] bytes, boxes {128, 128}; tm_out: out [N x K] bf16, boxes {32, 32}
+__global__ void k_merge_tc(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_a,
+                           const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_out,
+                           MergeParams p);
+constexpr int kMergeStages = 2;        // operand stages (one 64-rank chunk of B and A each)
+constexpr int kMergeCodeStages = 3;    // code tiles in flight
+constexpr int kMergeDrainWarps = 16;   // 4 lane quarters x 4 blocks of 64 columns
+constexpr size_t merge_tc_smem_bytes() {
+  return 1024 + kMergeStages * 49152 + kMergeCodeStages * 16384 + kMergeDrainWarps * 2 * 2048 + 256;
+}
 
 // AdamW step over n parameters (fp32 master, grad, m, v; optional bf16 copy).
 struct AdamwParams {

@@ -24,6 +24,8 @@
 //      one 16-byte store (fully coalesced along the row).
 #include "kernels.h"
 #include "nf4_dev.cuh"
+#include "ptx.cuh"
+#include "tc_common.cuh"
 
 namespace qlora {
 
@@ -228,6 +230,270 @@ __global__ void __launch_bounds__(256, 2) k_merge_lora(MergeParams p) {
       o[j] = pack_bf16x2(__fadd_rn(w0, d[2 * j]), __fadd_rn(w1, d[2 * j + 1]));
     }
     __stcs(reinterpret_cast<uint4*>(p.out + e0), make_uint4(o[0], o[1], o[2], o[3]));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core merge. Persistent CTAs (one per SM) walk 128-row x 256-column
+// output tiles (columns fastest). For each tile
+//   D[128 x 256] (fp32, tensor memory) = B[n0 .., 0 .. r64) A[0 .. r64, k0 ..)
+// runs on tcgen05 (M 128, N 256, K 16 per instruction), A and B arriving by
+// TMA in 64-rank chunks (B K-major, A MN-major, zero past r, N and K), while
+// the tile's packed codes arrive by TMA in a 128 x 128-byte swizzled box.
+// Sixteen drain warps (lane quarter w % 4, 64-column block (w - 2) / 4: one
+// weight block per row) then take 32 columns at a time: 32 accumulator
+// values per row from tensor memory (the next chunk's load in flight), 16
+// bytes of codes from shared memory, the block's 16-entry table (its scale
+// data fetched one tile ahead), w_hat = bf16(fl32(c[q] s_hat)) by table
+// lookup, one fp32 multiply by s, one fp32 add, one rounding, and a 32 x 32
+// TMA store. Two accumulators let the drain of one tile overlap the
+// products of the next.
+//
+// Warps: 0 TMA producer (one lane), 1 tensor-memory owner and MMA issuer
+// (one lane), 2-17 drain. Every wait is bounded; every TMA load fills only
+// this CTA's shared memory.
+__global__ void __launch_bounds__(576, 1)
+    k_merge_tc(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_a,
+               const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_out,
+               MergeParams p) {
+  using namespace tcd;
+  constexpr int STAGES = kMergeStages;
+  constexpr int CST = kMergeCodeStages;
+  constexpr uint32_t B_BYTES = 16384;          // 128 rows of B x 64 ranks (MMA operand A, K-major)
+  constexpr uint32_t A_BYTES = 32768;          // 64 ranks x 256 columns of A (MMA operand B, MN-major)
+  constexpr uint32_t STAGE_BYTES = B_BYTES + A_BYTES;
+  constexpr uint32_t C_BYTES = 16384;          // 128 rows x 128 bytes of codes
+  constexpr uint32_t IDESC = idesc_bf16_f32(128, 256, false, true);
+  constexpr uint32_t ACC_COLS = 256;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t codes0 = base + STAGES * STAGE_BYTES;
+  const uint32_t epi0 = codes0 + CST * C_BYTES;         // two 2 KB boxes per drain warp
+  const uint32_t bar0 = epi0 + kMergeDrainWarps * 2 * 2048;
+  uint8_t* const ctl = smem_raw + (bar0 - raw);
+  auto bar_full = [&](int s) { return bar0 + 8u * s; };
+  auto bar_empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto bar_cfull = [&](int c) { return bar0 + 8u * (2 * STAGES + c); };
+  auto bar_cempty = [&](int c) { return bar0 + 8u * (2 * STAGES + CST + c); };
+  auto bar_accf = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * CST + b); };
+  auto bar_acce = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * CST + 2 + b); };
+  const uint32_t bar_fin = bar0 + 8u * (2 * STAGES + 2 * CST + 4);
+  uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(ctl + 8 * (2 * STAGES + 2 * CST + 5));
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(ctl + 8 * (2 * STAGES + 2 * CST + 5) + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ntiles = p.tiles_n * p.tiles_k;
+  const int nchunks = p.r64 / 64;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int c = 0; c < CST; ++c) {
+      mbar_init(bar_cfull(c), 1);
+      mbar_init(bar_cempty(c), kMergeDrainWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf(b), 1);
+      mbar_init(bar_acce(b), kMergeDrainWarps);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 2 * ACC_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_b);
+      tma_prefetch_desc(&tm_a);
+      tma_prefetch_desc(&tm_codes);
+      int it = 0, i = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++i) {
+        const int n0 = (tile / p.tiles_k) * 128;
+        const int k0 = (tile % p.tiles_k) * 256;
+        const int cs = i % CST;
+        if (!mbar_wait(bar_cempty(cs), ((i / CST) & 1) ^ 1, abort_flag, QLORA_DEV_TIMEOUT_PRODUCER)) break;
+        const uint32_t c_s = codes0 + cs * C_BYTES;
+        mbar_arrive_expect_tx(bar_cfull(cs), C_BYTES);
+        tma_load_2d(c_s, &tm_codes, bar_cfull(cs), k0 / 2, n0);
+        for (int c = 0; c < nchunks; ++c, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(bar_empty(s), ((it / STAGES) & 1) ^ 1, abort_flag, QLORA_DEV_TIMEOUT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          const uint32_t b_s = base + s * STAGE_BYTES;
+          const uint32_t a_s = b_s + B_BYTES;
+          mbar_arrive_expect_tx(bar_full(s), STAGE_BYTES);
+          tma_load_2d(b_s, &tm_b, bar_full(s), c * 64, n0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) tma_load_2d(a_s + j * 8192, &tm_a, bar_full(s), k0 + 64 * j, c * 64);
+        }
+      }
+      // every load this thread started has landed before the CTA can exit
+      for (int j = max(0, it - STAGES); j < it; ++j) drain_wait(bar_full(j % STAGES), (j / STAGES) & 1);
+      for (int j = max(0, i - CST); j < i; ++j) drain_wait(bar_cfull(j % CST), (j / CST) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int it = 0, i = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++i) {
+        const int b = i & 1;
+        if (!mbar_wait(bar_acce(b), ((i >> 1) & 1) ^ 1, abort_flag, QLORA_DEV_TIMEOUT_MMA)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + b * ACC_COLS;
+        for (int c = 0; c < nchunks; ++c, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(bar_full(s), (it / STAGES) & 1, abort_flag, QLORA_DEV_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b_s = base + s * STAGE_BYTES;
+          const uint32_t a_s = b_s + B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t da = smem_desc_sw128(b_s + kk * 32, 16, 1024);
+            const uint64_t db = smem_desc_sw128(a_s + kk * 2048, 8192, 1024);
+            tc_mma_ss(d_tmem, da, db, IDESC, (c > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(bar_empty(s));
+        }
+        if (ok) tc_commit(bar_accf(b));
+      }
+      tc_commit(bar_fin);
+      drain_wait(bar_fin, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- drain
+    const int quarter = warp & 3;          // tensor-memory lanes [32 quarter, +32)
+    const int cb = (warp - 2) >> 2;        // columns [64 cb, +64) of the tile: one block per row
+    const int row = quarter * 32 + lane;   // this lane's row of the tile
+    const int64_t kpr = p.k >> 6;          // blocks per weight row
+    const uint32_t box0 = epi0 + (warp - 2) * 4096;
+    // raw scale data of this lane's block in a tile (zero past N or K)
+    struct ScaleData {
+      uint32_t q2;
+      float c0, c1;
+    };
+    auto fetch_scale = [&](int tile) {
+      ScaleData d{0u, 0.0f, 0.0f};
+      if (tile < ntiles) {
+        const int64_t n = (tile / p.tiles_k) * 128 + row;
+        const int64_t kc = (tile % p.tiles_k) * 256 + 64 * cb;
+        if (n < p.n && kc < p.k) {
+          const int64_t blk = n * kpr + (kc >> 6);
+          if (!p.dq) {
+            d.c0 = __ldg(p.smax + blk);
+          } else if (p.dqc == 2) {
+            d.q2 = __ldg(p.q2 + blk);
+            d.c0 = __ldg(p.smax + 2 * (blk >> 8));
+            d.c1 = __ldg(p.smax + 2 * (blk >> 8) + 1);
+          } else {
+            d.q2 = __ldg(p.q2 + blk);
+            d.c0 = __ldg(p.smax + (blk >> 8));
+          }
+        }
+      }
+      return d;
+    };
+    int i = 0, nbox = 0;
+    ScaleData nxt = fetch_scale(blockIdx.x);
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+      const int n0 = (tile / p.tiles_k) * 128;
+      const int k0 = (tile % p.tiles_k) * 256;
+      const ScaleData cur = nxt;
+      nxt = fetch_scale(tile + gridDim.x);   // in flight while this tile drains
+      const float sh = p.dq ? dq_block_scale(cur.q2, cur.c0, cur.c1, p.dqc) : cur.c0;
+      const int cs = i % CST;
+      const int b = i & 1;
+      bool ok = mbar_wait(bar_cfull(cs), (i / CST) & 1, abort_flag, QLORA_DEV_TIMEOUT_EPI);
+      if (ok) ok = mbar_wait(bar_accf(b), (i >> 1) & 1, abort_flag, QLORA_DEV_TIMEOUT_EPI);
+      if (!warp_all(ok)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + b * ACC_COLS + (static_cast<uint32_t>(quarter * 32) << 16) + 64 * cb;
+      const uint32_t crow = codes0 + cs * C_BYTES + row * 128;
+      const Nf4Table tb = make_table(p.cb, sh);
+      const uint64_t s2 = f2(p.s, p.s);
+      uint32_t acc0[32], acc1[32];
+      tmem_ld_32x32b_x32(taddr, acc0);
+      tmem_ld_32x32b_x32(taddr + 32, acc1);
+      const uint4 cw0 = lds128(crow + ((((cb << 1) + 0) ^ (row & 7)) << 4));
+      const uint4 cw1 = lds128(crow + ((((cb << 1) + 1) ^ (row & 7)) << 4));
+      tc_wait_ld();
+      // every accumulator column and code word of this warp is in registers
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar_acce(b));
+        mbar_arrive(bar_cempty(cs));
+      }
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        const uint32_t* acc = ch ? acc1 : acc0;
+        const uint4 cw = ch ? cw1 : cw0;
+        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+        uint32_t o[16];
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) {
+          uint32_t wh[4];
+          lookup8(tb, words[wd], wh);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            // (w_hat + fl32(s * acc)) for both weights of the pair at once
+            const uint64_t d2 = f2_mul(s2, f2(__uint_as_float(acc[8 * wd + 2 * j]),
+                                              __uint_as_float(acc[8 * wd + 2 * j + 1])));
+            uint32_t y0, y1;
+            f2_split(f2_add(f2(__uint_as_float(wh[j] << 16), __uint_as_float(wh[j] & 0xFFFF0000u)), d2), y0, y1);
+            o[4 * wd + j] = pack_bf16x2(__uint_as_float(y0), __uint_as_float(y1));
+          }
+        }
+        const int x = k0 + 64 * cb + 32 * ch;
+        if (x < p.k) {
+          // stage the 32 x 32 chunk (64-byte swizzle) in the box the store
+          // before last used, once that store has read it, and store it
+          const uint32_t box = box0 + (nbox & 1) * 2048;
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+          __syncwarp();
+          const uint32_t rw = box + lane * 64;
+          const uint32_t sw = (lane >> 1) & 3;
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            sts128(rw + ((v ^ sw) << 4), o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_out, box, x, n0 + quarter * 32);
+            bulk_commit();
+          }
+          ++nbox;
+        }
+      }
+    }
+    if (lane == 0) bulk_wait_all();   // stores complete before the CTA's shared memory goes away
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * ACC_COLS);
   }
 }
 

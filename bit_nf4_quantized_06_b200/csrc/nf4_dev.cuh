@@ -44,6 +44,24 @@ __device__ __forceinline__ float dq_block_scale(uint32_t q2, float c0, float c1,
   return restored_scale(q2, c0);
 }
 
+// Block-scale format as a compile-time constant, for kernels instantiated
+// per format: no double quantization (fp32 block scales), or one of the
+// three scale codes (qlora_dq_code_t + 1).
+constexpr int kScNone = 0, kScU8x256 = 1, kScU8x255 = 2, kScS8Mid = 3;
+
+__host__ __device__ constexpr int scale_format(int dq, int dqc) { return dq ? dqc + 1 : kScNone; }
+
+// Restored block scale for format SC: c0 is the fp32 block scale (kScNone)
+// or the group constant (s_max, or mid for kScS8Mid with c1 = half).
+template <int SC>
+__device__ __forceinline__ float block_scale_sc(uint32_t q2, float c0, float c1) {
+  if constexpr (SC == kScNone) {
+    return c0;
+  } else {
+    return dq_block_scale(q2, c0, c1, SC - 1);
+  }
+}
+
 // cb: the 16 fp32 levels (kernel-parameter constants).
 __device__ __forceinline__ Nf4Table make_table(const float (&cb)[16], float s_hat) {
   uint32_t p[8];

@@ -49,6 +49,13 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
   return v;
 }
 
+// 8-byte shared-memory load (cell entry: midpoint, count of midpoints below + 1)
+__device__ __forceinline__ uint2 lds_u2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
@@ -92,14 +99,14 @@ __device__ __noinline__ uint32_t exact_code(float w, float s, const double* cut)
 // around a large constant) selects the one level midpoint m inside the cell
 // (a cell is narrower than the gaps between midpoints) and the number of
 // midpoints below it, so q = below + [x' > m] -- exactly the count
-// #{j : fl32(w / s) > m_j} whenever |x' - m| exceeds the guard. The work runs
-// on the floating-point pipe: [x' > m] is a saturated product
-// sat(d * 2^100) of d = x' - m (0 or 1), the near-midpoint test the sum over
-// the chunk of sat(G^2 - d^2) (positive when some |d| < G), and the eight
-// codes are packed into the 32-bit word by exact float multiply-adds
-// (integers below 2^16) read back through the 2^23 offset. The two 33-word
-// tables sit one word per bank, so the lookups never conflict; each is read
-// at 4 bits(t) + constant, t the cell's float. Chunks with a
+// #{j : fl32(w / s) > m_j} whenever |x' - m| exceeds the guard. Two weights
+// go through each step as a packed fp32 pair (mul / fma .f32x2, each lane
+// rounded like the scalar operation): x', the cell's float t, and d^2 - G^2
+// whose sign bit says |d| < G for d = x' - m. One 8-byte table entry per
+// cell holds m and (midpoints below + 1); the word is the sum of those counts
+// at the eight nibble positions minus the sign bits of the eight d's (x' < m
+// takes one off), gathered with byte permutes -- d is never zero here, as
+// |d| >= G > 0. The table is read at 8 bits(t) + constant. Chunks with a
 // quotient within the guard of a midpoint take the exact test above for
 // those weights; blocks whose scale is zero, subnormal, at least 2^126 or not
 // finite take it (or the value the definition gives) for every weight.
@@ -108,6 +115,7 @@ __global__ void __launch_bounds__(256, 3) k_quantize_nf4(const uint4* __restrict
                                                       uint8_t* __restrict__ q2,
                                                       float* __restrict__ smax, QuantParams qp) {
   __shared__ float s_tab[66];     // [0, 33): the midpoint in each cell; [33, 66): midpoints below it
+  __shared__ uint2 s_cell[33];    // per cell: (bits of its midpoint, midpoints below it + 1)
   __shared__ double s_cut[16];
   __shared__ uint32_t s_wmax[8];
   __shared__ uint32_t s_wmin[8];
@@ -126,6 +134,7 @@ __global__ void __launch_bounds__(256, 3) k_quantize_nf4(const uint4* __restrict
   if (tid < 33) {
     s_tab[tid] = qp.cell_m[tid];
     s_tab[33 + tid] = qp.cell_below[tid];
+    s_cell[tid] = make_uint2(__float_as_uint(qp.cell_m[tid]), static_cast<uint32_t>(qp.cell_below[tid]) + 1u);
   }
   if (tid < 16) s_cut[tid] = qp.cut[tid];
 
@@ -203,6 +212,7 @@ __global__ void __launch_bounds__(256, 3) k_quantize_nf4(const uint4* __restrict
   constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: the integer part lands in the low mantissa bits
   // shared address of cell c's midpoint is 4 * bits(t) + tab_base, t = 16 x + 16 + kMagic
   const uint32_t tab_base = smem_u32(s_tab) - __float_as_uint(kMagic) * 4u;
+  const uint32_t cell_base = smem_u32(s_cell) - __float_as_uint(kMagic) * 8u;   // cell c at 8 c
   constexpr float kGuard2 = kEncodeGuard * kEncodeGuard;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -216,27 +226,41 @@ __global__ void __launch_bounds__(256, 3) k_quantize_nf4(const uint4* __restrict
       uint32_t word = 0;
       bool slow = edge;
       if (!edge) {
+        // two weights per step: bf16 pair h holds element 2h (low half, high
+        // nibble of byte h) and element 2h + 1 (high half, low nibble)
         const float r = rcp_approx(sb);
-        float qf[8];
-        float amb = 0.0f;
+        const uint64_t r2 = f2(r, r);
+        const uint64_t k16 = f2(16.0f, 16.0f), kc = f2(16.0f + kMagic, 16.0f + kMagic);
+        const uint64_t ng2 = f2(-kGuard2, -kGuard2);
+        uint32_t dev[4], dod[4];   // bits of x - m for the even and the odd element of each pair
+        uint32_t near = 0, bsum = 0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          // element e of the chunk: bf16 pair e/2 holds element 2k in its low half
-          const float we = (e & 1) ? __uint_as_float(ww[e >> 1] & 0xFFFF0000u) : __uint_as_float(ww[e >> 1] << 16);
-          const float x = __fmul_rn(we, r);
-          const float t = fmaf(x, 16.0f, 16.0f + kMagic);   // cell 0..32: |x| <= 1 + 2^-21
-          const uint32_t addr = __float_as_uint(t) * 4u + tab_base;
-          const float d = __fsub_rn(x, lds_f32(addr));
-          qf[e] = __fadd_rn(lds_f32(addr + 132u), __saturatef(__fmul_rn(d, 0x1p100f)));
-          amb = __fadd_rn(amb, __saturatef(fmaf(-d, d, kGuard2)));
+        for (int h = 0; h < 4; ++h) {
+          const uint64_t x2 = f2_mul(f2(__uint_as_float(ww[h] << 16), __uint_as_float(ww[h] & 0xFFFF0000u)), r2);
+          uint32_t t0, t1, x0, x1;
+          f2_split(f2_fma(x2, k16, kc), t0, t1);        // cells 0..32: |x| <= 1 + 2^-21
+          f2_split(x2, x0, x1);
+          const uint2 c0 = lds_u2(t0 * 8u + cell_base);
+          const uint2 c1 = lds_u2(t1 * 8u + cell_base);
+          const float d0 = __fsub_rn(__uint_as_float(x0), __uint_as_float(c0.x));
+          const float d1 = __fsub_rn(__uint_as_float(x1), __uint_as_float(c1.x));
+          dev[h] = __float_as_uint(d0);
+          dod[h] = __float_as_uint(d1);
+          // d^2 - G^2 < 0 (sign bit set) exactly when |d| < G
+          uint32_t g0, g1;
+          f2_split(f2_fma(f2(d0, d1), f2(d0, d1), ng2), g0, g1);
+          near |= g0 | g1;
+          // each nibble first gets (midpoints below + 1); the code is one less
+          // where x is below the cell's midpoint (d < 0)
+          bsum += c0.y * (16u << (8 * h)) + c1.y * (1u << (8 * h));
         }
-        if (amb > 0.0f) {
+        if (near & 0x80000000u) {
           slow = true;
         } else {
-          // byte j holds element 2j in its high nibble: word = lo + 2^16 hi
-          const float lo = __fadd_rn(fmaf(qf[2], 4096.0f, fmaf(qf[3], 256.0f, fmaf(qf[0], 16.0f, qf[1]))), 8388608.0f);
-          const float hi = __fadd_rn(fmaf(qf[6], 4096.0f, fmaf(qf[7], 256.0f, fmaf(qf[4], 16.0f, qf[5]))), 8388608.0f);
-          word = __float_as_uint(hi) * 65536u + __float_as_uint(lo) - 0x4B000000u;
+          // sign bits of d: even elements to bits 8h + 4, odd ones to bits 8h
+          const uint32_t se = prmt(prmt(dev[0], dev[1], 0x0073u), prmt(dev[2], dev[3], 0x7300u), 0x7610u);
+          const uint32_t so = prmt(prmt(dod[0], dod[1], 0x0073u), prmt(dod[2], dod[3], 0x7300u), 0x7610u);
+          word = bsum - ((se >> 3) & 0x10101010u) - ((so >> 7) & 0x01010101u);
         }
       }
       if (slow) {

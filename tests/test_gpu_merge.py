@@ -34,10 +34,15 @@ def _ulps(a_bits, b_bits):
 
 CASES = [
     # n, k, r, alpha, outliers, b_scale
+    # r % 8 == 0: the tensor-core merge (128 x 256 tiles)
     (256, 256, 8, 16.0, False, 1.0),
-    (200, 192, 12, 16.0, False, 30.0),     # ragged rows and k-tiles, r not a multiple of 8, visible adapter
+    (128, 512, 256, 16.0, False, 5.0),     # largest rank: four 64-rank chunks per tile
+    (200, 192, 16, 16.0, False, 30.0),     # ragged rows, one partial column tile
+    (300, 320, 96, 32.0, True, 10.0),      # ragged rows, second column tile 64 wide, two chunks
+    (1000, 1344, 64, 16.0, True, 10.0),    # 8 x 6 tiles over 148 CTAs, last column tile half full
+    # r % 8 != 0: the element-wise merge
+    (200, 192, 12, 16.0, False, 30.0),     # ragged rows and k-tiles, visible adapter
     (384, 1024, 100, 32.0, True, 10.0),
-    (128, 512, 256, 16.0, False, 5.0),     # largest rank
 ]
 
 
