@@ -642,7 +642,9 @@ int current_sms() {
 
 size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r) {
   if (m < 0 || n_out <= 0 || k_in <= 0 || r < 1 || r > kMaxRank) return 0;
-  return plan_ws(std::max<int64_t>(m, 1), n_out, k_in, r, current_sms(), false, g_sched.load()).sk_total;
+  // sized for the stream-K slots wherever any schedule setting could use
+  // them, so the answer does not depend on the process-wide setting
+  return plan_ws(std::max<int64_t>(m, 1), n_out, k_in, r, current_sms(), false, QLORA_SCHED_STREAM_K).sk_total;
 }
 
 size_t qlora_fwd_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r) {

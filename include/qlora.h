@@ -152,13 +152,13 @@ QLORA_API qlora_status_t qlora_quantize_nf4(const void *w_bf16, const qlora_nf4_
 QLORA_API qlora_status_t qlora_dequantize(const qlora_nf4_t *q, void *w_bf16_out, void *stream);
 
 /* Workspace bytes for qlora_linear_fwd / _bwd at these sizes: covers both
- * calls, every forward path, and, where the GEMM schedule
- * (qlora_set_gemm_schedule) would use stream-K, its fp32 partial slots (up to
- * 256 KB per SM). 0 for arguments out of range. The size depends on the SM
- * count of the current device and on the schedule setting: ask with the
- * device current that the calls will run on. A smaller workspace, down to
- * what qlora_fwd_workspace_bytes reports for the forward, is accepted; the
- * GEMMs then run data-parallel. */
+ * calls, every forward path, and the stream-K schedule's fp32 partial slots
+ * (up to 256 KB per SM) wherever some setting of qlora_set_gemm_schedule
+ * could run stream-K, so the answer does not change with that setting. 0 for
+ * arguments out of range. The size depends on the SM count of the current
+ * device: ask with the device current that the calls will run on. A smaller
+ * workspace, down to what qlora_fwd_workspace_bytes reports for the
+ * forward, is accepted; the GEMMs then run data-parallel. */
 QLORA_API size_t qlora_workspace_bytes(int64_t m, int64_t n_out, int64_t k_in, int32_t r);
 
 /* The least workspace that qlora_linear_fwd accepts for these sizes (at most
