@@ -54,6 +54,17 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 
 __device__ __forceinline__ float bf16_round_f(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
+// fl32(w + c) for the bf16 in the low (hi = 0) or high half of `pair`: the
+// bf16 operand widens exactly, so this is the fp32 sum rounded to nearest even
+__device__ __forceinline__ float add_bf16_f32(uint32_t pair, float c, int hi) {
+  float d;
+  if (hi)
+    asm("{ .reg .b16 l, h; mov.b32 {l, h}, %1; add.rn.f32.bf16 %0, h, %2; }" : "=f"(d) : "r"(pair), "f"(c));
+  else
+    asm("{ .reg .b16 l, h; mov.b32 {l, h}, %1; add.rn.f32.bf16 %0, l, %2; }" : "=f"(d) : "r"(pair), "f"(c));
+  return d;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(256, 2) k_merge_lora(MergeParams p) {
@@ -456,12 +467,13 @@ __global__ void __launch_bounds__(576, 1)
           lookup8(tb, words[wd], wh);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            // (w_hat + fl32(s * acc)) for both weights of the pair at once
-            const uint64_t d2 = f2_mul(s2, f2(__uint_as_float(acc[8 * wd + 2 * j]),
-                                              __uint_as_float(acc[8 * wd + 2 * j + 1])));
-            uint32_t y0, y1;
-            f2_split(f2_add(f2(__uint_as_float(wh[j] << 16), __uint_as_float(wh[j] & 0xFFFF0000u)), d2), y0, y1);
-            o[4 * wd + j] = pack_bf16x2(__uint_as_float(y0), __uint_as_float(y1));
+            // fl32(s * acc) for both weights of the pair at once, then
+            // w_hat + that with the bf16 w_hat widened inside the add
+            uint32_t d0, d1;
+            f2_split(f2_mul(s2, f2(__uint_as_float(acc[8 * wd + 2 * j]), __uint_as_float(acc[8 * wd + 2 * j + 1]))),
+                     d0, d1);
+            o[4 * wd + j] = pack_bf16x2(add_bf16_f32(wh[j], __uint_as_float(d0), 0),
+                                        add_bf16_f32(wh[j], __uint_as_float(d1), 1));
           }
         }
         const int x = k0 + 64 * cb + 32 * ch;
