@@ -12,7 +12,7 @@ Functions carry the C names:
     qlora_workspace_bytes, qlora_fwd_workspace_bytes, qlora_linear_fwd, qlora_linear_fwd_ex,
     qlora_linear_fwd_noalloc, qlora_linear_bwd, qlora_device_status, qlora_status_string, qlora_version,
     qlora_launch_count, qlora_selftest_wait_timeout, qlora_merge_lora, qlora_adamw_step, qlora_adamw_host,
-    qlora_adamw_paged, qlora_set_gemm_schedule, qlora_get_gemm_schedule
+    qlora_adamw_paged, qlora_adamw_staged, qlora_set_gemm_schedule, qlora_get_gemm_schedule
 """
 
 import ctypes
@@ -25,7 +25,7 @@ __all__ = [
     "qlora_linear_bwd",
     "qlora_device_status", "qlora_status_string", "qlora_version", "qlora_launch_count",
     "qlora_selftest_wait_timeout", "qlora_merge_lora", "qlora_adamw_step", "qlora_adamw_host", "qlora_adamw_paged",
-    "qlora_set_gemm_schedule", "qlora_get_gemm_schedule",
+    "qlora_adamw_staged", "qlora_set_gemm_schedule", "qlora_get_gemm_schedule",
     "AdamwParams",
     "FWD_AUTO", "FWD_GEMM", "FWD_GEMV", "SCHED_AUTO", "SCHED_DATA_PARALLEL", "SCHED_STREAM_K",
 ]
@@ -103,6 +103,8 @@ lib.qlora_adamw_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, ctypes.POINTER(A
 lib.qlora_adamw_host.restype = ctypes.c_int
 lib.qlora_adamw_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, ctypes.POINTER(AdamwParams), _vp]
 lib.qlora_adamw_paged.restype = ctypes.c_int
+lib.qlora_adamw_staged.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, ctypes.POINTER(AdamwParams), _vp]
+lib.qlora_adamw_staged.restype = ctypes.c_int
 lib.qlora_merge_lora.argtypes = [_P(Nf4Struct), _vp, _vp, _i32, _f32, _vp, _vp]
 lib.qlora_merge_lora.restype = ctypes.c_int
 lib.qlora_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _vp]
@@ -354,6 +356,20 @@ def qlora_adamw_step(master, grad, m, v, step, lr=1e-4, betas=(0.9, 0.999), eps=
     hp = AdamwParams(float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay), int(step))
     _check(lib.qlora_adamw_step(_ptr(master), _ptr(param) if param is not None else None, _ptr(grad), _ptr(m),
                                 _ptr(v), n, ctypes.byref(hp), _stream_ptr(stream)), "qlora_adamw_step")
+
+
+def qlora_adamw_staged(master, grad, m_host, v_host, m_stage, v_stage, step, lr=1e-4, betas=(0.9, 0.999),
+                       eps=1e-8, weight_decay=0.0, param=None, stream=None):
+    """One AdamW step with m, v in pinned host memory, staged through the
+    device buffers m_stage, v_stage by copies on `stream` (H2D, update, D2H)."""
+    n = master.numel()
+    for t in (grad, m_host, v_host, m_stage, v_stage) + ((param,) if param is not None else ()):
+        if t.numel() != n:
+            raise ValueError("qlora_adamw_staged: element counts differ")
+    hp = AdamwParams(float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay), int(step))
+    _check(lib.qlora_adamw_staged(_ptr(master), _ptr(param) if param is not None else None, _ptr(grad),
+                                  _ptr(m_host), _ptr(v_host), _ptr(m_stage), _ptr(v_stage), n, ctypes.byref(hp),
+                                  _stream_ptr(stream)), "qlora_adamw_staged")
 
 
 def qlora_adamw_host(master, grad, m, v, step, lr=1e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0,

@@ -7,6 +7,7 @@
 #include <cstring>
 #include <atomic>
 #include <mutex>
+#include <utility>
 
 #include <cudaTypedefs.h>
 
@@ -335,16 +336,19 @@ inline bool sk_wanted(int64_t kt_main, int mode) {
 struct WsPlan {
   size_t u_pad, v_pad, b_pad, dy_pad, part, total;
   bool sk_ok;        // a pair GEMM of the call may use the stream-K schedule
-  size_t sk_total;   // total with room for the stream-K slots (>= total)
+  size_t sk_total;   // total with room for the stream-K slots and flags (>= total)
+  size_t flags_off;  // stream-K flags (sk_total plan), from the 256-aligned workspace start
 };
 
-// Workspace layout: [u_pad][v_pad][b_pad][dy_pad][split partials], each
-// 256-aligned. The forward needs no v_pad, no dy_pad and only the x A^T
+// Workspace layout: [u_pad][v_pad][b_pad][dy_pad][split partials][flags],
+// each 256-aligned. The forward needs no v_pad, no dy_pad and only the x A^T
 // partials. dy_pad holds dY with its rows padded to a multiple of 8 elements
 // when N % 8 != 0 (the TMA loads of dY need 16-byte row strides). The pair kernels'
 // stream-K slots reuse the partials region (it is free while they run), which
-// grows to hold them in the sk_total plan: `total` is what a call needs,
-// `sk_total` what lets it use the stream-K schedule when that pays.
+// grows to hold them in the sk_total plan; their flags get a region of their
+// own, zeroed at the start of the call, before any kernel of the call runs:
+// `total` is what a call needs, `sk_total` what lets it use the stream-K
+// schedule when that pays.
 WsPlan plan_ws(int64_t m, int64_t n, int64_t k, int32_t r, int sms, bool fwd_only, int mode) {
   const int32_t r64 = r64_of(r);
   WsPlan w{};
@@ -363,9 +367,9 @@ WsPlan plan_ws(int64_t m, int64_t n, int64_t k, int32_t r, int sms, bool fwd_onl
   // the forward reduces over K, dX over N; slots only where stream-K may run
   const int64_t tiles = std::max(sk_wanted(cdiv(k, 64), mode) ? pair_tiles(m, n) : int64_t(0),
                                  fwd_only || !sk_wanted(cdiv(n, 64), mode) ? int64_t(0) : pair_tiles(m, k));
-  const size_t sk = al256(sk_part_bytes(m, sms)) + al256(sk_flag_bytes(sms));
   w.sk_ok = m > kGemvMaxM && tiles > sms / 4;
-  w.sk_total = w.sk_ok ? w.total - w.part + std::max(w.part, sk) : w.total;
+  w.flags_off = w.u_pad + w.v_pad + w.b_pad + w.dy_pad + std::max(w.part, al256(sk_part_bytes(m, sms)));
+  w.sk_total = w.sk_ok ? w.flags_off + al256(sk_flag_bytes(sms)) + 256 : w.total;
   return w;
 }
 
@@ -397,6 +401,38 @@ CUtensorMap zero_map() {
   return m;
 }
 
+// Launch as a programmatic dependent of the kernel in front on the stream:
+// the kernel itself waits for that grid before touching global memory (every
+// kernel launched this way calls grid_dependency_wait first), so stream order
+// holds while the launch and the kernel's set-up overlap the one in front.
+template <typename... KArgs, typename... Args>
+qlora_status_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+// Zero-padded copy of a [rows x r] bf16 matrix into [rows x r64].
+qlora_status_t pad_cols(const __nv_bfloat16* src, __nv_bfloat16* dst, int64_t rows, int32_t r, int32_t r64, int sms,
+                        cudaStream_t st) {
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(cdiv(rows * r64, 256), int64_t(sms) * 8));
+  return launch_pdl(k_pad_cols, dim3(std::max(blocks, 1u)), dim3(256), 0, st, src, dst, rows, r, r64);
+}
+
 // Persistent launch: one CTA per SM at most, each walking the tile list.
 template <int BN, int AS, int BS>
 qlora_status_t launch_small_bn(int sms, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& b,
@@ -404,8 +440,8 @@ qlora_status_t launch_small_bn(int sms, cudaStream_t st, const CUtensorMap& a, c
   const int64_t tiles = static_cast<int64_t>(p.tiles) * p.splits;
   if (tiles <= 0) return QLORA_ERR_SHAPE;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, sms));
-  k_tc_small<BN, AS, BS, small_stages(BN)><<<grid, 192, tc_small_smem_bytes<BN>(), st>>>(a, b, p);
-  return launch_status();
+  return launch_pdl(k_tc_small<BN, AS, BS, small_stages(BN)>, dim3(grid), dim3(192), tc_small_smem_bytes<BN>(), st,
+                    a, b, p);
 }
 
 // Persistent CTA-pair launch: at most `pairs` clusters of two CTAs.
@@ -416,17 +452,21 @@ qlora_status_t launch_pair_nh(int pairs, cudaStream_t st, const CUtensorMap& b, 
   if (tiles <= 0 || pairs <= 0) return QLORA_ERR_SHAPE;
   const unsigned nclusters = static_cast<unsigned>(std::min<int64_t>(tiles, pairs));
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // a programmatic dependent of the kernel in front (the pair kernel waits
+  // for it before touching global memory)
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(2 * nclusters, 1, 1);
   cfg.blockDim = dim3(448, 1, 1);
   cfg.dynamicSmemBytes = tc_pair_smem_bytes(NH);
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc_pair<AS, NH>, b, bl, c, o, p);
   if (e != cudaSuccess) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -458,12 +498,14 @@ int32_t pick_feat_n(int64_t features, int64_t tiles_cols, int pairs) {
 // stores when its row stride is a multiple of 16 bytes.
 //
 // Stream-K: with `sk_region` (the workspace's partials region, holding at
-// least the slots and flags of sk_part_bytes / sk_flag_bytes) and a tile
-// count above the pair count that leaves the last wave partly idle, the
-// pairs split the work evenly (see k_tc_pair); the flags are zeroed first.
+// least the slots of sk_part_bytes) and `sk_flags` (sk_flag_bytes, zeroed by
+// the caller before the call's first kernel), and a tile count above the
+// pair count that leaves the last wave partly idle, the pairs split the work
+// evenly (see k_tc_pair).
 template <int AS>
 qlora_status_t launch_pair(int pairs, int64_t m, cudaStream_t st, const CUtensorMap& b, const CUtensorMap& bl,
-                           const CUtensorMap& c, TcParams p, uint8_t* sk_region, int sms, int mode) {
+                           const CUtensorMap& c, TcParams p, uint8_t* sk_region, uint32_t* sk_flags, int sms,
+                           int mode) {
   CUtensorMap o = zero_map();
   p.tma_out = 0;
   if (p.ldo % 8 == 0 && (reinterpret_cast<uintptr_t>(p.out) & 15u) == 0) {
@@ -481,15 +523,11 @@ qlora_status_t launch_pair(int pairs, int64_t m, cudaStream_t st, const CUtensor
   p.sk = 0;
   p.sk_part = nullptr;
   p.sk_flags = nullptr;
-  if (sk_region != nullptr && sk_wanted(p.kt_main, mode) && p.tma_out && pairs > 1 && 2 * pairs <= sms &&
-      tiles > pairs && tiles % pairs != 0) {
+  if (sk_region != nullptr && sk_flags != nullptr && sk_wanted(p.kt_main, mode) && p.tma_out && pairs > 1 &&
+      2 * pairs <= sms && tiles > pairs && tiles % pairs != 0) {
     p.sk = 1;
     p.sk_part = reinterpret_cast<float*>(sk_region);
-    p.sk_flags = reinterpret_cast<uint32_t*>(sk_region + al256(sk_part_bytes(m, sms)));
-    if (cudaMemsetAsync(p.sk_flags, 0, sk_flag_bytes(sms), st) != cudaSuccess) {
-      cudaGetLastError();
-      return QLORA_ERR_CUDA;
-    }
+    p.sk_flags = sk_flags;
   }
   if (AS == A_DQ_K && !p.sk && pairs > 0) {
     p.feat_n = pick_feat_n(p.rows, p.tiles_cols, pairs);
@@ -540,8 +578,7 @@ qlora_status_t lora_product(const CUtensorMap& ma, const CUtensorMap& mb, int64_
   if (s != QLORA_OK) return s;
   const int total = p.rows * (r64 / 4);
   const int blocks = static_cast<int>(std::min<int64_t>(cdiv(total, 256), int64_t(sms) * 8));
-  k_reduce_splits<<<std::max(blocks, 1), 256, 0, st>>>(p);
-  return launch_status();
+  return launch_pdl(k_reduce_splits, dim3(std::max(blocks, 1)), dim3(256), 0, st, p);
 }
 
 struct LinearArgs {
@@ -724,10 +761,18 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
   const auto* bb = static_cast<const __nv_bfloat16*>(b);
   const __nv_bfloat16* b_use = bb;
   int64_t ldb = r;
+  // stream-K flags, zeroed before the call's first kernel (the chain of
+  // kernels below runs as programmatic dependents, with no memset between)
+  uint32_t* sk_flags = nullptr;
+  if (path == QLORA_FWD_GEMM && wp.sk_ok && ws_bytes >= wp.sk_total) {
+    sk_flags = reinterpret_cast<uint32_t*>(wsb + wp.flags_off);
+    if (cudaMemsetAsync(sk_flags, 0, sk_flag_bytes(sms), st) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+  }
   if (r % 8 != 0) {
-    k_pad_cols<<<static_cast<unsigned>(std::min<int64_t>(cdiv(n * r64, 256), int64_t(sms) * 8)), 256, 0, st>>>(
-        bb, b_pad, n, r, r64);
-    if ((s = launch_status()) != QLORA_OK) return s;
+    if ((s = pad_cols(bb, b_pad, n, r, r64, sms, st)) != QLORA_OK) return s;
     b_use = b_pad;
     ldb = r64;
   }
@@ -839,8 +884,7 @@ qlora_status_t qlora_linear_fwd_ex(const qlora_nf4_t* q, const void* x, int64_t 
   p.out = y;
   p.ldo = n;
   return launch_pair<A_DQ_K>(pairs, m, st, m_x_b, m_u, m_codes, p,
-                             wp.sk_ok && ws_bytes >= wp.sk_total ? reinterpret_cast<uint8_t*>(part) : nullptr, sms,
-                             mode);
+                             sk_flags != nullptr ? reinterpret_cast<uint8_t*>(part) : nullptr, sk_flags, sms, mode);
 }
 
 qlora_status_t qlora_linear_fwd(const qlora_nf4_t* q, const void* x, int64_t m, const void* a, const void* b,
@@ -886,20 +930,27 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
   const auto* ab = static_cast<const __nv_bfloat16*>(a);
   const auto* bb = static_cast<const __nv_bfloat16*>(b);
   const auto* dyb = static_cast<const __nv_bfloat16*>(dy);
+  // stream-K flags, zeroed before the call's first kernel (the chain of
+  // kernels below runs as programmatic dependents, with no memset between)
+  uint32_t* sk_flags = nullptr;
+  if (dx != nullptr && wp.sk_ok && ws_bytes >= wp.sk_total) {
+    sk_flags = reinterpret_cast<uint32_t*>(wsb + wp.flags_off);
+    if (cudaMemsetAsync(sk_flags, 0, sk_flag_bytes(sms), st) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+  }
   // dY rows reach the tensor maps with a 16-byte stride: pad them when N % 8 != 0
   const int64_t ldn = rup(n, 8);
   if (ldn != n) {
-    k_pad_cols<<<static_cast<unsigned>(std::min<int64_t>(cdiv(m * ldn, 256), int64_t(sms) * 8)), 256, 0, st>>>(
-        dyb, dy_pad, m, static_cast<int32_t>(n), static_cast<int32_t>(ldn));
-    if ((s = launch_status()) != QLORA_OK) return s;
+    if ((s = pad_cols(dyb, dy_pad, m, static_cast<int32_t>(n), static_cast<int32_t>(ldn), sms, st)) != QLORA_OK)
+      return s;
     dyb = dy_pad;
   }
   const __nv_bfloat16* b_use = bb;
   int64_t ldb = r;
   if (r % 8 != 0) {
-    k_pad_cols<<<static_cast<unsigned>(std::min<int64_t>(cdiv(n * r64, 256), int64_t(sms) * 8)), 256, 0, st>>>(
-        bb, b_pad, n, r, r64);
-    if ((s = launch_status()) != QLORA_OK) return s;
+    if ((s = pad_cols(bb, b_pad, n, r, r64, sms, st)) != QLORA_OK) return s;
     b_use = b_pad;
     ldb = r64;
   }
@@ -911,9 +962,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
     u_use = static_cast<const __nv_bfloat16*>(u);
     ldu = r;
   } else if (u != nullptr) {
-    k_pad_cols<<<static_cast<unsigned>(std::min<int64_t>(cdiv(m * r64, 256), int64_t(sms) * 8)), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(u), u_pad, m, r, r64);
-    if ((s = launch_status()) != QLORA_OK) return s;
+    if ((s = pad_cols(static_cast<const __nv_bfloat16*>(u), u_pad, m, r, r64, sms, st)) != QLORA_OK) return s;
     u_use = u_pad;
   } else {
     CUtensorMap m_x_a, m_at;
@@ -965,8 +1014,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
     p.out = dx;
     p.ldo = k;
     s = launch_pair<A_DQ_MN>(pairs, m, st, m_dy_b, m_v, m_codes, p,
-                             wp.sk_ok && ws_bytes >= wp.sk_total ? reinterpret_cast<uint8_t*>(part) : nullptr, sms,
-                             mode);
+                             sk_flags != nullptr ? reinterpret_cast<uint8_t*>(part) : nullptr, sk_flags, sms, mode);
     if (s != QLORA_OK) return s;
   }
 
@@ -1039,22 +1087,54 @@ qlora_status_t qlora_merge_lora(const qlora_nf4_t* q, const void* a, const void*
   return launch_status();
 }
 
-qlora_status_t qlora_adamw_step(float* master, void* param_bf16, const float* grad, float* m, float* v, int64_t n,
-                                const qlora_adamw_t* hp, void* stream) {
+namespace {
+// Argument checks of the AdamW entry points (nothing enqueued yet).
+qlora_status_t check_adamw(const float* master, const void* param_bf16, const float* grad, const float* m,
+                           const float* v, int64_t n, const qlora_adamw_t* hp) {
   if (hp == nullptr || n < 0) return QLORA_ERR_INVALID_ARG;
   if (n == 0) return QLORA_OK;
   if (master == nullptr || grad == nullptr || m == nullptr || v == nullptr) return QLORA_ERR_INVALID_ARG;
   if (hp->step < 1 || !(hp->lr >= 0.0f) || !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) ||
       !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) || !(hp->eps > 0.0f) || !std::isfinite(hp->weight_decay))
     return QLORA_ERR_INVALID_ARG;
-  const auto a4 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if ((reinterpret_cast<uintptr_t>(master) | reinterpret_cast<uintptr_t>(grad) | reinterpret_cast<uintptr_t>(m) |
        reinterpret_cast<uintptr_t>(v)) & 3u)
     return QLORA_ERR_ALIGNMENT;
   if (param_bf16 != nullptr && (reinterpret_cast<uintptr_t>(param_bf16) & 1u)) return QLORA_ERR_ALIGNMENT;
+  return QLORA_OK;
+}
+}  // namespace
+
+qlora_status_t qlora_adamw_staged(float* master, void* param_bf16, const float* grad, float* m_host, float* v_host,
+                                  float* m_stage, float* v_stage, int64_t n, const qlora_adamw_t* hp, void* stream) {
+  qlora_status_t s = check_adamw(master, param_bf16, grad, m_stage, v_stage, n, hp);
+  if (s != QLORA_OK || n == 0) return s;
+  if (m_host == nullptr || v_host == nullptr) return QLORA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(m_host) | reinterpret_cast<uintptr_t>(v_host)) & 3u) return QLORA_ERR_ALIGNMENT;
+  if ((s = device_ready(nullptr)) != QLORA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(n) * sizeof(float);
+  if (cudaMemcpyAsync(m_stage, m_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(v_stage, v_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  if ((s = qlora_adamw_step(master, param_bf16, grad, m_stage, v_stage, n, hp, stream)) != QLORA_OK) return s;
+  if (cudaMemcpyAsync(m_host, m_stage, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(v_host, v_stage, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  return QLORA_OK;
+}
+
+qlora_status_t qlora_adamw_step(float* master, void* param_bf16, const float* grad, float* m, float* v, int64_t n,
+                                const qlora_adamw_t* hp, void* stream) {
+  qlora_status_t s = check_adamw(master, param_bf16, grad, m, v, n, hp);
+  if (s != QLORA_OK || n == 0) return s;
+  const auto a4 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   int sms = 0;
-  qlora_status_t s = device_ready(&sms);
-  if (s != QLORA_OK) return s;
+  if ((s = device_ready(&sms)) != QLORA_OK) return s;
   AdamwParams a{};
   a.master = master;
   a.grad = grad;

@@ -44,11 +44,6 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return v;
 }
 
-// Programmatic dependent launch: the consumer waits for the producer grid's
-// completion (and memory) only where it reads the producer's output.
-__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dependency_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 __device__ __forceinline__ uint32_t ld_bf16_pair(const __nv_bfloat16* row, int j, int r) {
   // (row[j], row[j+1]) with zeros past r; 2-byte loads so any r works
   const uint16_t* p = reinterpret_cast<const uint16_t*>(row);

@@ -345,6 +345,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool a_mn_ma
          | ((uint32_t)(m >> 4) << 24);
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched as a programmatic dependent of the one before it on the
+// stream may start while that one finishes: it waits for the earlier grid's
+// completion (and memory) before it touches global memory, then lets the
+// next launch start. Where every kernel of a chain does this in that order,
+// the chain keeps stream order while the launches and set-up overlap.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ packed fp32 pairs
 // Two fp32 lanes in one 64-bit register pair: packed multiply, add and fused
 // multiply-add (each lane rounded to nearest even exactly as the scalar op).

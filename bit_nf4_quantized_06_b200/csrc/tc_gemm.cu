@@ -91,6 +91,10 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // launched as a programmatic dependent: the set-up above overlapped the
+  // kernel in front; its results are visible from here on
+  grid_dependency_wait();
+  grid_dependency_trigger();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -217,6 +221,8 @@ __global__ void __launch_bounds__(192, 1)
 // Each thread handles four consecutive columns of one row; for mode 2 rows
 // run fastest across threads so that the transposed writes coalesce.
 __global__ void __launch_bounds__(256) k_reduce_splits(SmallParams p) {
+  grid_dependency_wait();
+  grid_dependency_trigger();
   const int q4 = p.ld >> 2;
   const int total = p.rows * q4;
   const int64_t slab = static_cast<int64_t>(p.rows_pad) * p.ld;
@@ -265,6 +271,8 @@ __global__ void __launch_bounds__(256) k_reduce_splits(SmallParams p) {
 __global__ void __launch_bounds__(256) k_pad_cols(const __nv_bfloat16* __restrict__ src,
                                                   __nv_bfloat16* __restrict__ dst, int64_t rows,
                                                   int32_t r, int32_t r64) {
+  grid_dependency_wait();
+  grid_dependency_trigger();
   const int64_t total = rows * r64;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;

@@ -137,6 +137,10 @@ __global__ void __launch_bounds__(448, 1)
   cluster_sync_all();   // barriers initialised and tensor memory allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // launched as a programmatic dependent: the set-up above overlapped the
+  // kernel in front; its results are visible from here on
+  grid_dependency_wait();
+  grid_dependency_trigger();
 
   // tile -> first feature of this CTA's restored slice, first token of the tile
   auto tile_feat = [&](int tile) { return (tile / p.tiles_cols) * FN + (FN >> 1) * static_cast<int>(rank); };

@@ -283,6 +283,21 @@ QLORA_API qlora_status_t qlora_adamw_paged(const float *grad_dev, void *param_de
                                            void *param_host_bf16, int64_t n, const qlora_adamw_t *hp,
                                            void *stream);
 
+/* AdamW with m and v kept in pinned host memory and staged through device
+ * memory (the paged optimizer with the copy engines doing the paging): on
+ * `stream`, copy m_host, v_host (pinned, n fp32 each) into m_stage, v_stage
+ * (device, n fp32 each, caller-owned scratch), run qlora_adamw_step on the
+ * staged states, and copy them back. The transfers hold no SMs, so issued on
+ * a second stream the update overlaps the kernels of other streams; two
+ * such streams used in turn overlap the host-to-device and device-to-host
+ * copies of consecutive updates. master, grad, param_bf16 as in
+ * qlora_adamw_step (device). Arguments are checked before anything is
+ * enqueued; m_stage and v_stage must not be in use by other work meanwhile.
+ * Results are bit-identical to qlora_adamw_step on device-resident states. */
+QLORA_API qlora_status_t qlora_adamw_staged(float *master, void *param_bf16, const float *grad, float *m_host,
+                                            float *v_host, float *m_stage, float *v_stage, int64_t n,
+                                            const qlora_adamw_t *hp, void *stream);
+
 /* Synchronises `stream`, then reads and clears the device status word of the
  * current device. Returns QLORA_OK, QLORA_ERR_TIMEOUT (a kernel gave up on a
  * bounded wait; *bits, if non-NULL, gets which role), or QLORA_ERR_CUDA. */

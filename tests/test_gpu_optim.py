@@ -75,3 +75,43 @@ def test_paged_chain_matches_oracle(q):
         assert np.allclose(master_h.double().numpy(), po, rtol=1e-6, atol=1e-5 * HP["lr"])
         rb = bf16.round_f32_to_bf16_bits(master_h.numpy())
         assert np.array_equal(param_d.cpu().view(torch.int16).numpy().view(np.uint16), rb)
+
+
+@pytest.mark.parametrize("n,offset", [(966656, 0), (1001, 1)])
+def test_staged_states_match_device_states_bit_for_bit(q, n, offset):
+    # m, v in pinned host memory staged through device buffers by copies on
+    # the stream: the same kernel on the same values as device-resident states
+    g = torch.Generator().manual_seed(5 * n + offset)
+    p0 = torch.randn(n + offset, generator=g) * 0.02
+    master_a, master_b = p0.clone().cuda(), p0.clone().cuda()
+    m_d, v_d = torch.zeros(n + offset, device="cuda"), torch.zeros(n + offset, device="cuda")
+    m_h, v_h = torch.zeros(n + offset).pin_memory(), torch.zeros(n + offset).pin_memory()
+    m_s, v_s = torch.empty(n + offset, device="cuda"), torch.empty(n + offset, device="cuda")
+    pa = torch.empty(n + offset, dtype=torch.bfloat16, device="cuda")
+    pb = torch.empty(n + offset, dtype=torch.bfloat16, device="cuda")
+    side = torch.cuda.Stream()
+    for t in range(1, 4):
+        grad = (torch.randn(n + offset, generator=g) * 0.01).cuda()
+        q.qlora_adamw_step(master_a[offset:], grad[offset:], m_d[offset:], v_d[offset:], t, param=pa[offset:], **HP)
+        side.wait_stream(torch.cuda.current_stream())
+        q.qlora_adamw_staged(master_b[offset:], grad[offset:], m_h[offset:], v_h[offset:], m_s[offset:],
+                             v_s[offset:], t, param=pb[offset:], stream=side, **HP)
+        side.synchronize()
+        torch.cuda.synchronize()
+        assert torch.equal(master_a, master_b)
+        assert torch.equal(m_d.cpu(), m_h) and torch.equal(v_d.cpu(), v_h)
+        assert torch.equal(pa.view(torch.int16), pb.view(torch.int16))
+    assert q.qlora_device_status() == (0, 0)
+
+
+def test_staged_rejects_bad_arguments_before_enqueueing(q):
+    n = 64
+    master = torch.zeros(n, device="cuda")
+    grad = torch.zeros(n, device="cuda")
+    m_h, v_h = torch.zeros(n).pin_memory(), torch.zeros(n).pin_memory()
+    m_s, v_s = torch.empty(n, device="cuda"), torch.empty(n, device="cuda")
+    with pytest.raises(q.QloraError):
+        q.qlora_adamw_staged(master, grad, m_h, v_h, m_s, v_s, 0)          # step must be >= 1
+    with pytest.raises(q.QloraError):
+        q.qlora_adamw_staged(master, grad, m_h, v_h, m_s, v_s, 1, eps=0.0)
+    assert torch.equal(m_h, torch.zeros(n))
