@@ -142,3 +142,49 @@ def test_backward_cut_tiles_restore_w_exactly(q):
     dx, _, _ = q.qlora_linear_bwd(qw, x.cuda(), None, dy.cuda(), a.cuda(), b.cuda(), 16.0, ws=_ws(q, n, n, k, r))
     torch.cuda.synchronize()
     assert np.array_equal(_bits(dx), nf4.dequantize_bits(o["codes"], o["q2"], o["smax"]))
+
+
+def test_fwd_bwd_in_cuda_graph_match_direct_calls(q):
+    # a forward and a backward call (each a chain of programmatic dependent
+    # launches; the stream-K flags zeroed by a memset before the chain)
+    # captured in one CUDA graph and replayed with new inputs: bit-identical to
+    # direct calls every time, so the flags start at zero on every replay and
+    # every kernel of the chain sees its predecessor's results
+    n, k, m, r, alpha = 2560, 128, 4096, 64, 16.0
+    qw = q.qlora_quantize_nf4(synth.weight(n, k, seed=21).cuda())
+    a = synth.lora_a(r, k, seed=22).cuda()
+    b = (synth.lora_b(n, r, seed=23).float() * 20).to(torch.bfloat16).cuda()
+    x = torch.empty((m, k), dtype=torch.bfloat16, device="cuda")
+    dy = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    u = torch.empty((m, r), dtype=torch.bfloat16, device="cuda")
+    dx = torch.empty((m, k), dtype=torch.bfloat16, device="cuda")
+    da = torch.empty((r, k), dtype=torch.float32, device="cuda")
+    db = torch.empty((n, r), dtype=torch.float32, device="cuda")
+    ws = _ws(q, m, n, k, r)
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        q.qlora_linear_fwd(qw, x, a, b, alpha, y=y, u=u, ws=ws, stream=st)
+    st.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        q.qlora_linear_fwd(qw, x, a, b, alpha, y=y, u=u, ws=ws, stream=st)
+        q.qlora_linear_bwd(qw, x, u, dy, a, b, alpha, dx=dx, da=da, db=db, ws=ws, stream=st)
+    for trial in range(3):
+        x.copy_(synth.tokens(m, k, seed=300 + trial))
+        dy.copy_(synth.grad_out(m, n, seed=400 + trial))
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        y2, u2 = q.qlora_linear_fwd(qw, x, a, b, alpha)
+        dx2, da2, db2 = q.qlora_linear_bwd(qw, x, u2, dy, a, b, alpha)
+        torch.cuda.synchronize()
+        assert torch.equal(_bits_t(y), _bits_t(y2)) and torch.equal(_bits_t(u), _bits_t(u2))
+        assert torch.equal(_bits_t(dx), _bits_t(dx2))
+        assert torch.equal(da, da2) and torch.equal(db, db2)
+    del g
+
+
+def _bits_t(t):
+    return t.view(torch.int16)
