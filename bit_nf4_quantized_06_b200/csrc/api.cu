@@ -610,7 +610,7 @@ using namespace qlora;
 
 extern "C" {
 
-int32_t qlora_version(void) { return 10100; }
+int32_t qlora_version(void) { return 10200; }
 
 uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 

@@ -118,7 +118,7 @@ struct TcParams {
   // the (tile, k-tile) space per CTA pair; a tile cut between two pairs goes
   // through one fp32 partial slot per CTA, [128 x 256 NH] floats each, laid
   // out [column / 4][row][4], and four ready flags per CTA (one per epilogue
-  // warp), zeroed before the launch
+  // warp), zeroed before the call's first kernel
   int32_t sk;
   float* sk_part;
   uint32_t* sk_flags;

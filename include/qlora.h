@@ -358,7 +358,7 @@ QLORA_API const char *qlora_status_string(qlora_status_t s);
 QLORA_API uint64_t qlora_launch_count(void);
 
 /* Library version as major*10000 + minor*100 + patch (1.1.0: qlora_nf4_t
- * gained dq_code and reserved). */
+ * gained dq_code and reserved; 1.2.0: qlora_adamw_staged). */
 QLORA_API int32_t qlora_version(void);
 
 #ifdef __cplusplus

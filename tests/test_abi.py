@@ -159,4 +159,4 @@ def test_nf4_bytes_of_the_scale_codes(q):
     assert q.lib.qlora_dequantize(ctypes.byref(s), ctypes.c_void_p(16), None) == 1
     s = q.Nf4Struct(512, 512, 64, 256, 16, 16, 16, 0, 1)
     assert q.lib.qlora_dequantize(ctypes.byref(s), ctypes.c_void_p(16), None) == 1
-    assert q.qlora_version() == 10100
+    assert q.qlora_version() == 10200
