@@ -40,6 +40,7 @@ CASES = [
     (200, 192, 16, 16.0, False, 30.0),     # ragged rows, one partial column tile
     (300, 320, 96, 32.0, True, 10.0),      # ragged rows, second column tile 64 wide, two chunks
     (1000, 1344, 64, 16.0, True, 10.0),    # 8 x 6 tiles over 148 CTAs, last column tile half full
+    (130, 64, 16, 16.0, False, 30.0),      # one 64-weight block per row: three of four drain blocks idle
     # r % 8 != 0: the element-wise merge
     (200, 192, 12, 16.0, False, 30.0),     # ragged rows and k-tiles, visible adapter
     (384, 1024, 100, 32.0, True, 10.0),
