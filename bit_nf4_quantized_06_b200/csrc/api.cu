@@ -902,20 +902,21 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
   if ((s = device_ready(&sms, &pairs)) != QLORA_OK) return s;
   const LinearArgs la{q, m, r, alpha, ws, ws_bytes};
   if ((s = check_linear(la, sms, false)) != QLORA_OK) return s;
-  if (x == nullptr || dy == nullptr || a == nullptr || b == nullptr || da == nullptr || db == nullptr)
-    return QLORA_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(dy) || !aligned16(a) || !aligned16(b) || !aligned16(da) || !aligned16(db) ||
-      (dx && !aligned16(dx)) || (u && !aligned16(u)))
-    return QLORA_ERR_ALIGNMENT;
+  if (da == nullptr || db == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(da) || !aligned16(db)) return QLORA_ERR_ALIGNMENT;
   const int64_t n = q->n_out, k = q->k_in;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (m == 0) {
-    // no tokens: the gradients are exactly zero
+    // no tokens (x, u, dY, A, B and dX are not read): the gradients are exactly zero
     if (cudaMemsetAsync(da, 0, static_cast<size_t>(r) * k * sizeof(float), st) != cudaSuccess ||
         cudaMemsetAsync(db, 0, static_cast<size_t>(n) * r * sizeof(float), st) != cudaSuccess)
       return QLORA_ERR_CUDA;
     return QLORA_OK;
   }
+  if (x == nullptr || dy == nullptr || a == nullptr || b == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(a) || !aligned16(b) || (dx && !aligned16(dx)) ||
+      (u && !aligned16(u)))
+    return QLORA_ERR_ALIGNMENT;
   const int32_t r64 = r64_of(r);
   const float sc = alpha / static_cast<float>(r);
   const int mode = g_sched.load();

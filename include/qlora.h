@@ -221,7 +221,9 @@ QLORA_API qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t *q, const vo
  * dB [N x r] fp32 (overwritten, not accumulated). u_bf16 is the u' that the
  * forward produced ([m x r], may be NULL: then it is recomputed). No gradient
  * into W. Any N: when N % 8 != 0 the call first copies dY into the workspace
- * with its rows padded to a multiple of 8 (qlora_workspace_bytes counts it). */
+ * with its rows padded to a multiple of 8 (qlora_workspace_bytes counts it).
+ * m == 0: dA and dB are set to zero; x, u, dY, A, B and dX are not read
+ * (they may be NULL) and no workspace is needed. */
 QLORA_API qlora_status_t qlora_linear_bwd(const qlora_nf4_t *q, const void *x_bf16, const void *u_bf16,
                                 const void *dy_bf16, int64_t m, const void *a_bf16,
                                 const void *b_bf16, int32_t r, float alpha, void *dx_bf16,

@@ -329,6 +329,21 @@ def test_forward_empty_tokens_is_noop(q):
     assert y.shape == (0, n)
 
 
+def test_backward_empty_tokens_gives_zero_gradients(q):
+    # no tokens: dA and dB are exactly zero (overwritten, whatever they held)
+    n, k, r = 128, 128, 8
+    qw = q.qlora_quantize_nf4(synth.weight(n, k).cuda())
+    x = torch.empty((0, k), dtype=torch.bfloat16, device="cuda")
+    dy = torch.empty((0, n), dtype=torch.bfloat16, device="cuda")
+    da = torch.full((r, k), 7.0, device="cuda")
+    db = torch.full((n, r), -3.0, device="cuda")
+    q.qlora_linear_bwd(qw, x, None, dy, synth.lora_a(r, k).cuda(), synth.lora_b(n, r).cuda(), 16.0, dx=None,
+                       da=da, db=db, ws=torch.empty(256, dtype=torch.uint8, device="cuda"), want_dx=False)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(da).item() == 0 and torch.count_nonzero(db).item() == 0
+    assert q.qlora_device_status() == (0, 0)
+
+
 # --------------------------------------------------------------------------- backward
 
 BWD_CASES = [
@@ -380,6 +395,8 @@ def test_backward_dx_restores_w_exactly(q):
 # multiples, so its epilogue stores each row directly instead of through TMA
 # boxes; the backward copies dY into row-padded workspace first
 ODD_N_CASES = [
+    (1, 128, 40, 8),         # a single output feature (dY padded from 1 to 8 columns)
+    (7, 64, 300, 16),        # fewer features than one restore slice, one k-tile
     (1001, 512, 300, 16),
     (37, 192, 64, 8),
     (100, 128, 16, 8),       # 16 tokens through the GEMM path
