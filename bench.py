@@ -1039,9 +1039,8 @@ def run_reference(args):
     a = t["a"].float().numpy().astype(np.float64)
     b = t["b"].float().numpy().astype(np.float64)
     dy = t["dy"].float().numpy().astype(np.float64)
-    tok = 32   # bounded sample of each step: full quantize + restore, fwd+bwd on 32 tokens
 
-    def step():
+    def step(tok):
         t0 = time.perf_counter()
         o = nf4.quantize(w)
         w_hat = nf4.dequantize(o["codes"], o["q2"], o["smax"]).astype(np.float64)
@@ -1050,28 +1049,45 @@ def run_reference(args):
         linear.backward(x[:tok], dy[:tok], w_hat, a, b, p.scale)
         return t1 - t0, time.perf_counter() - t1
 
-    for _ in range(args.warmup):
-        step()
+    # Each step is the full quantize + restore and fp64 fwd+bwd on as many of
+    # the 4096 tokens as keep the whole run (warm-up and timed steps) within
+    # about 150 s on these cores: all of them where the cores allow, so that
+    # the step is the GPU arm's workload itself. The first warm-up step
+    # measures the rates (256 tokens).
+    budget_s = 150.0
+    tq0, tf0 = step(256)
+    remaining = max(1, args.steps + args.warmup - 1)
+    per_tok = tf0 / 256
+    tok = int((budget_s / remaining - tq0) / per_tok) // 32 * 32
+    tok = max(32, min(p.m, tok))
+    for _ in range(args.warmup - 1):
+        step(tok)
     tq = tf = 0.0
     for _ in range(args.steps):
-        a_, b_ = step()
+        a_, b_ = step(tok)
         tq += a_
         tf += b_
     tq /= args.steps
     tf /= args.steps
     dt = tq + tf
     # the same rate as the GPU arm's: the step's fwd+bwd flops at 4096 tokens
-    # over the quantize time plus the sampled fwd+bwd time scaled to 4096 tokens
+    # over the quantize time plus the fwd+bwd time (scaled to 4096 tokens
+    # when fewer were run)
     full = tq + tf * p.m / tok
     value = (fwd_flops(p.m, p.n, p.k, p.r) + bwd_flops(p.m, p.n, p.k, p.r)) / full / 1e12
-    sample = (f"numpy oracle per step: quantize+restore the full 11008x4096 W ({tq:.2f} s), fp64 fwd+bwd on "
-              f"{tok} of 4096 tokens ({tf:.2f} s); rate over the step scaled to 4096 tokens ({full:.1f} s)")
+    if tok == p.m:
+        sample = (f"numpy oracle per step: quantize+restore the full 11008x4096 W ({tq:.2f} s), fp64 fwd+bwd on "
+                  f"all 4096 tokens ({tf:.2f} s): the GPU arm's step")
+        wl = p.name + " fwd+bwd with its quantize (the full step)"
+    else:
+        sample = (f"numpy oracle per step: quantize+restore the full 11008x4096 W ({tq:.2f} s), fp64 fwd+bwd on "
+                  f"{tok} of 4096 tokens ({tf:.2f} s); rate over the step scaled to 4096 tokens ({full:.1f} s)")
+        wl = p.name + " fwd+bwd (bounded token sample) with its quantize"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": p.name + " fwd+bwd (bounded token sample) with its quantize", "tokens_per_step": tok,
-                   "extrapolated_full_step_ms": round(full * 1e3, 1)},
+        "config": {"workload": wl, "tokens_per_step": tok, "full_step_ms": round(full * 1e3, 1)},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
