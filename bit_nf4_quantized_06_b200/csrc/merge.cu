@@ -10,8 +10,10 @@
 //
 // The pass is bound by HBM: it reads 0.5 byte of codes (plus 1/64 byte of
 // scale code) and writes 2 bytes of bf16 per weight, while the rank-r product
-// costs 2 r flops per weight and runs on the tensor cores. One CTA owns a
-// 128 x 128 tile of the output:
+// costs 2 r flops per weight and runs on the tensor cores. Two kernels:
+// k_merge_tc (below; tcgen05, operands by TMA) when B's rows are 16-byte
+// aligned (r % 8 == 0), and k_merge_lora for the other ranks, where one CTA
+// owns a 128 x 128 tile of the output:
 //   1. B[n0 .. n0+128][0 .. r64) and A[0 .. r64)[k0 .. k0+128) are staged in
 //      shared memory (zero past r, N and K);
 //   2. eight warps (a 4 x 2 grid of 32 x 64 sub-tiles) form B A with
@@ -252,13 +254,14 @@ __global__ void __launch_bounds__(256, 2) k_merge_lora(MergeParams p) {
 // TMA in 64-rank chunks (B K-major, A MN-major, zero past r, N and K), while
 // the tile's packed codes arrive by TMA in a 128 x 128-byte swizzled box.
 // Sixteen drain warps (lane quarter w % 4, 64-column block (w - 2) / 4: one
-// weight block per row) then take 32 columns at a time: 32 accumulator
-// values per row from tensor memory (the next chunk's load in flight), 16
-// bytes of codes from shared memory, the block's 16-entry table (its scale
-// data fetched one tile ahead), w_hat = bf16(fl32(c[q] s_hat)) by table
-// lookup, one fp32 multiply by s, one fp32 add, one rounding, and a 32 x 32
-// TMA store. Two accumulators let the drain of one tile overlap the
-// products of the next.
+// weight block per row) load their 64 accumulator values per row from tensor
+// memory and their 32 bytes of codes from shared memory at once, release
+// both, and then per 32 columns: the block's 16-entry table (its scale data
+// fetched one tile ahead), w_hat = bf16(fl32(c[q] s_hat)) by table lookup,
+// fl32(s * acc) for two weights at a time, the add w_hat + that in fp32 (the
+// bf16 w_hat widens exactly inside the mixed-precision add), one rounding,
+// and a 32 x 32 TMA store. Two accumulators let the drain of one tile
+// overlap the products of the next.
 //
 // Warps: 0 TMA producer (one lane), 1 tensor-memory owner and MMA issuer
 // (one lane), 2-17 drain. Every wait is bounded; every TMA load fills only
