@@ -19,7 +19,9 @@
 // and both kernels use programmatic dependent launch: x A^T may launch while
 // the kernel before it drains, waits for it, and then lets the GEMV start;
 // the GEMV streams the whole weight while x A^T runs beside it and waits for
-// x A^T only before the LoRA-up step that reads u'.
+// x A^T only before the LoRA-up step that reads u'. The GEMV is instantiated
+// per block-scale format (no double quantization, or one of the three scale
+// codes), so the restore of one format carries no code for the others.
 #include "kernels.h"
 #include "nf4_dev.cuh"
 
