@@ -638,14 +638,93 @@ def whole_stack(q, device, l2):
         raise RuntimeError(f"device status {st} ({bits:#x}) in the stack sweep")
     fl = sum(fwd_flops(m, n, k, r) + bwd_flops(m, n, k, r) for _, n, k, _, _ in lin)
     qb = sum(quant_bytes(n, k) for _, n, k, _, _ in lin)
+    fused = stack_fused_siblings(q, lin, xs, m, r, alpha, l2, fl)
     popt = stack_paged_optimizer(q, lin, xs, dys, ys, dxs, ws, m, r, alpha, l2)
     del lin
     return {"weights": params, "linears": 224, "quantize_ms": round(q_ms, 3), "paged_optimizer": popt,
+            "fused_siblings": fused,
             "quantize_GB/s": round(qb / (q_ms * 1e-3) / 1e9, 1), "fwd_bwd_ms": round(t_ms, 3),
             "fwd_bwd_TFLOP": round(fl / 1e12, 2), "fwd_bwd_TFLOP/s": round(fl / (t_ms * 1e-3) / 1e12, 1),
             "fwd_bwd_graph_ms": round(tg_ms, 3), "fwd_bwd_graph_TFLOP/s": round(fl / (tg_ms * 1e-3) / 1e12, 1),
             "workload": "whole 7B-shaped stack, 32 x (q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008), "
                         "4096 tokens, r=64, weights generated on the GPU per layer"}
+
+
+def concat_nf4(q, parts):
+    """The packed weight of parts' matrices stacked along d_out: the codes,
+    scale codes and group constants concatenate (blocks lie within rows, and
+    each part's row count times its blocks per row is a whole number of
+    256-block groups), so no re-quantization is needed."""
+    n = sum(p.n_out for p in parts)
+    out = q.NF4Weight(n, parts[0].k_in, device=parts[0].codes.device)
+    for name in ("codes", "scale_codes", "absmax"):
+        torch.cat([getattr(p, name) for p in parts], out=getattr(out, name))
+    return out
+
+
+def stack_fused_siblings(q, lin, xs, m, r, alpha, l2, fl):
+    """The whole stack's fwd+bwd with sibling projections fused, as a
+    deployment would run it: per layer one call for q, k, v (12288 x 4096,
+    adapters stacked to r = 192, B block diagonal) and one for gate, up
+    (22016 x 4096, r = 128), o and down as before. Same algorithmic FLOPs as
+    the 224 separate linears; one event pair around the sweep, L2 flushed
+    first."""
+    dev = xs[4096].device
+    per_layer = len(synth.STACK7B_LAYER)
+    groups = []
+    for layer in range(synth.STACK7B_LAYERS):
+        lp = lin[layer * per_layer:(layer + 1) * per_layer]
+        for idx in ((0, 1, 2), (3,), (4, 5), (6,)):
+            parts = [lp[i] for i in idx]
+            if len(parts) == 1:
+                qw, n, k, a, b = parts[0]
+                groups.append((qw, n, k, a, b, alpha, r))
+                continue
+            qc = concat_nf4(q, [p_[0] for p_ in parts])
+            n = sum(p_[1] for p_ in parts)
+            k = parts[0][2]
+            rr = r * len(parts)
+            a_cat = torch.cat([p_[3] for p_ in parts], 0)
+            b_bd = torch.zeros((n, rr), dtype=torch.bfloat16, device=dev)
+            row = 0
+            for j, p_ in enumerate(parts):
+                b_bd[row:row + p_[1], j * r:(j + 1) * r] = p_[4]
+                row += p_[1]
+            groups.append((qc, n, k, a_cat, b_bd, alpha * len(parts), rr))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(synth.STACK7B_ACT_SEED + 1)
+    dys = {n: torch.randn((m, n), generator=gen, device=dev).to(torch.bfloat16) for n in (4096, 11008, 12288, 22016)}
+    ys = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in dys}
+    dxs = {k: torch.empty((m, k), dtype=torch.bfloat16, device=dev) for k in (4096, 11008)}
+    us = {rr: torch.empty((m, rr), dtype=torch.bfloat16, device=dev) for rr in (r, 2 * r, 3 * r)}
+    das = {(rr, k): torch.empty((rr, k), dtype=torch.float32, device=dev) for rr in (r, 2 * r, 3 * r)
+           for k in (4096, 11008)}
+    dbs = {(n, rr): torch.empty((n, rr), dtype=torch.float32, device=dev) for n in dys for rr in (r, 2 * r, 3 * r)}
+    wsz = max(q.qlora_workspace_bytes(m, n, k, rr) for _, n, k, _, _, _, rr in groups)
+    ws = torch.empty(wsz + 256, dtype=torch.uint8, device=dev)
+
+    def sweep():
+        for qw, n, k, a, b, al, rr in groups:
+            q.qlora_linear_fwd(qw, xs[k], a, b, al, y=ys[n], u=us[rr], ws=ws)
+            q.qlora_linear_bwd(qw, xs[k], us[rr], dys[n], a, b, al, dx=dxs[k], da=das[(rr, k)], db=dbs[(n, rr)],
+                               ws=ws)
+
+    sweep()
+    flush_l2(l2)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    sweep()
+    e1.record()
+    torch.cuda.synchronize()
+    t_ms = e0.elapsed_time(e1)
+    st, bits = q.qlora_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({bits:#x}) in the fused stack sweep")
+    return {"calls": 2 * len(groups), "fwd_bwd_ms": round(t_ms, 3),
+            "fwd_bwd_TFLOP/s": round(fl / (t_ms * 1e-3) / 1e12, 1),
+            "workload": "the same stack with q,k,v fused (12288x4096, r=192) and gate,up fused (22016x4096, r=128) "
+                        "per layer; o and down separate; FLOPs counted as for the separate linears"}
 
 
 def stack_paged_optimizer(q, lin, xs, dys, ys, dxs, ws, m, r, alpha, l2, steps=3):
