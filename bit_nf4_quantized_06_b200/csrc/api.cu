@@ -552,7 +552,8 @@ qlora_status_t launch_small(int32_t r64, int sms, cudaStream_t st, const CUtenso
 // A TMA-fed LoRA product over a reduction of length `kdim`: split-K partial
 // slabs in `part`, then the fixed-order reduction writes mode 0 bf16(scale *
 // .) to out_pad [rows x r64] (and out_c [rows x r] when set), mode 1 fp32
-// out_f [rows x r], mode 2 fp32 out_f [r x rows] (transposed).
+// out_f [rows x r], mode 2 fp32 out_f [r x rows] (transposed). With one
+// split the GEMM's drain writes the result and no reduction is launched.
 template <int AS, int BS>
 qlora_status_t lora_product(const CUtensorMap& ma, const CUtensorMap& mb, int64_t rows, int64_t kdim,
                             int32_t r, float scale, int mode, __nv_bfloat16* out_pad, __nv_bfloat16* out_c,
@@ -575,7 +576,7 @@ qlora_status_t lora_product(const CUtensorMap& ma, const CUtensorMap& mb, int64_
   p.out_c = out_c;
   p.out_f = out_f;
   qlora_status_t s = launch_small<AS, BS>(r64, sms, st, ma, mb, p);
-  if (s != QLORA_OK) return s;
+  if (s != QLORA_OK || p.splits == 1) return s;   // one split: the GEMM wrote the result itself
   const int total = p.rows * (r64 / 4);
   const int blocks = static_cast<int>(std::min<int64_t>(cdiv(total, 256), int64_t(sms) * 8));
   return launch_pdl(k_reduce_splits, dim3(std::max(blocks, 1)), dim3(256), 0, st, p);
@@ -983,6 +984,15 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
     if (s != QLORA_OK) return s;
   }
 
+  // dB [N x r] = dY^T u'  (A = dY seen MN-major, B = u' MN-major), right after
+  // dY B so that much of dY is still in L2 when it is read again
+  {
+    CUtensorMap m_dymn, m_umn;
+    if (!map_bf16(&m_dymn, dyb, m, n, ldn, 64) || !map_bf16(&m_umn, u_use, m, ldu == r ? r : r64, ldu, 64))
+      return QLORA_ERR_CUDA;
+    s = lora_product<A_TMA_MN, B_TMA_MN>(m_dymn, m_umn, n, m, r, 1.0f, 1, nullptr, nullptr, db, part, sms, st);
+    if (s != QLORA_OK) return s;
+  }
   // dX^T tiles: A = restored W seen MN-major (reduction over d_out), B = dY,
   // plus v' A_lora as extra k-tiles
   if (dx != nullptr) {
@@ -1024,14 +1034,6 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t* q, const void* x, const void*
     CUtensorMap m_xmn, m_vmn;
     if (!map_bf16(&m_xmn, xb, m, k, k, 64) || !map_bf16(&m_vmn, v_pad, m, r64, r64, 64)) return QLORA_ERR_CUDA;
     s = lora_product<A_TMA_MN, B_TMA_MN>(m_xmn, m_vmn, k, m, r, 1.0f, 2, nullptr, nullptr, da, part, sms, st);
-    if (s != QLORA_OK) return s;
-  }
-  // dB [N x r] = dY^T u'  (A = dY seen MN-major, B = u' MN-major)
-  {
-    CUtensorMap m_dymn, m_umn;
-    if (!map_bf16(&m_dymn, dyb, m, n, ldn, 64) || !map_bf16(&m_umn, u_use, m, ldu == r ? r : r64, ldu, 64))
-      return QLORA_ERR_CUDA;
-    s = lora_product<A_TMA_MN, B_TMA_MN>(m_dymn, m_umn, n, m, r, 1.0f, 1, nullptr, nullptr, db, part, sms, st);
     if (s != QLORA_OK) return s;
   }
   return QLORA_OK;

@@ -5,7 +5,8 @@
 // accumulators in tensor memory let the drain of tile i overlap the main
 // loop of tile i + 1. fp32 partial tiles go to a workspace slab per split
 // and a fixed-order reduction kernel finishes them (deterministic):
-// bf16(s * u) for x A^T and dY B, fp32 dA (transposed) and dB.
+// bf16(s * u) for x A^T and dY B, fp32 dA (transposed) and dB. Without a
+// split the drain writes those results itself and no reduction runs.
 //
 //   D[128 x BN] (fp32, tensor memory)  +=  A[128 x 64] * B[BN x 64]^T  per k-tile
 //
@@ -27,6 +28,38 @@ namespace {
 template <int BN>
 constexpr uint32_t tmem_cols() {
   return BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+}
+
+// The last step of the split reduction for columns [c0, c0 + 32) of output
+// row `row`, given their complete fp32 sums v (what k_reduce_splits does
+// after summing the slabs): mode 0 bf16(scale * v) to out_pad [rows x ld]
+// and out_c [rows x cols] (if set), mode 1 fp32 out_f [rows x cols], mode 2
+// fp32 out_f [cols x rows] (consecutive lanes hold consecutive rows, so the
+// transposed stores of a warp coalesce).
+__device__ __forceinline__ void finish_row(const SmallParams& p, int row, int c0, const uint32_t (&v)[32]) {
+  if (p.mode == 0) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * p.scale, __uint_as_float(v[2 * i + 1]) * p.scale);
+    uint4* dst = reinterpret_cast<uint4*>(p.out_pad + static_cast<int64_t>(row) * p.ld + c0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    if (p.out_c != nullptr) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (c0 + i < p.cols)
+          p.out_c[static_cast<int64_t>(row) * p.cols + c0 + i] = __float2bfloat16_rn(__uint_as_float(v[i]) * p.scale);
+    }
+  } else if (p.mode == 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (c0 + i < p.cols) p.out_f[static_cast<int64_t>(row) * p.cols + c0 + i] = __uint_as_float(v[i]) * p.scale;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (c0 + i < p.cols) p.out_f[static_cast<int64_t>(c0 + i) * p.rows + row] = __uint_as_float(v[i]) * p.scale;
+  }
 }
 
 }  // namespace
@@ -194,6 +227,12 @@ __global__ void __launch_bounds__(192, 1)
         if (empty) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = 0u;
+        }
+        if (p.splits == 1) {
+          // one split: this is the whole sum, so the reduction's final step
+          // (scale, convert, layout) is done here and no slab is written
+          if (prow < p.rows) finish_row(p, prow, ch * 32, r);
+          continue;
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i)

@@ -219,6 +219,11 @@ FWD_CASES = [
     (37, 64, 16, 8, "gemv"),         # one block per row, 16 tokens
     (8, 11008, 2, 64, "gemv"),       # eight rows, a long reduction
     (22016, 256, 1, 16, "gemv"),     # many row groups, short rows
+    # one 64-wide k-tile of x A^T (k = 64): the small GEMM runs unsplit and
+    # its drain writes u' (and the caller's u) itself, no reduction launch
+    (64, 64, 100, 16, "gemm"),
+    (136, 64, 40, 12, "gemm"),       # ... with r % 8 != 0 (padded u', narrow caller u)
+    (64, 64, 33, 128, "gemm"),       # ... with 128-column tiles
 ]
 
 
@@ -353,6 +358,11 @@ BWD_CASES = [
     (256, 256, 129, 100),
     (384, 1024, 513, 256),
     (1000, 512, 70, 12),
+    # unsplit small GEMMs whose drains write the results (one k-tile in the
+    # reduction): dA and dB (m <= 64), dY B (n = 64), x A^T when recomputed (k = 64)
+    (64, 64, 100, 16),
+    (136, 64, 40, 12),
+    (64, 64, 33, 128),
 ]
 
 
@@ -546,6 +556,67 @@ def test_decode_in_cuda_graph_sees_new_inputs(q):
             assert torch.equal(y1.view(torch.int16), r1.view(torch.int16))
             assert torch.equal(y2.view(torch.int16), r2.view(torch.int16))
         del g
+    assert q.qlora_device_status() == (0, 0)
+
+
+def test_decode_chain_reads_outputs_of_the_kernels_in_front(q):
+    # decode calls whose x is the output of the call just before (a GEMM-path
+    # forward first, then decode calls through two ping-pong buffers), queued
+    # back to back on one stream and once more as a CUDA graph: the decode
+    # kernels start streaming the packed weight while the kernels in front
+    # still run, so any read of x, B or u' before the kernels in front are
+    # complete would show here as a difference from the same chain run call
+    # by call with a synchronisation between the calls
+    n = k = 1024
+    r, alpha = 16, 16.0
+    qws = [q.qlora_quantize_nf4(synth.weight(n, k, seed=40 + i).cuda()) for i in range(2)]
+    a = synth.lora_a(r, k, seed=42).cuda()
+    b = (synth.lora_b(n, r, seed=43).float() * 30).to(torch.bfloat16).cuda()
+    x0 = synth.tokens(64, k, seed=44).cuda()
+    layers = 6
+
+    def chain(bufs, ws, st, sync):
+        y0, pp = bufs
+        q.qlora_linear_fwd(qws[0], x0, a, b, alpha, y=y0, ws=ws, want_u=False, stream=st)
+        src = y0[:1]
+        for i in range(layers):
+            if sync:
+                torch.cuda.synchronize()
+            dst = pp[i % 2]
+            q.qlora_linear_fwd(qws[(i + 1) % 2], src, a, b, alpha, y=dst, ws=ws, want_u=False, stream=st)
+            src = dst
+        return src
+
+    def buffers():
+        return (torch.empty((64, n), dtype=torch.bfloat16, device="cuda"),
+                [torch.full((1, n), float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(2)])
+
+    ws = torch.empty(q.qlora_workspace_bytes(64, n, k, r) + 256, dtype=torch.uint8, device="cuda")
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    ref_bufs = buffers()
+    with torch.cuda.stream(st):
+        ref = chain(ref_bufs, ws, st, sync=True).clone()
+    torch.cuda.synchronize()
+    assert torch.isfinite(ref.float()).all()
+    for _ in range(3):
+        bufs = buffers()
+        with torch.cuda.stream(st):
+            got = chain(bufs, ws, st, sync=False)
+        torch.cuda.synchronize()
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    bufs = buffers()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        got = chain(bufs, ws, st, sync=False)
+    for _ in range(3):
+        for t in bufs[1]:
+            t.fill_(float("nan"))
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    del g
     assert q.qlora_device_status() == (0, 0)
 
 
