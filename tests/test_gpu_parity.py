@@ -385,6 +385,30 @@ def test_backward_parity(q, n, k, m, r, with_u):
     assert linear.rel_fro(_np(db), db_ref) <= TOL
 
 
+@pytest.mark.parametrize("n,k,m,r", [(1024, 512, 300, 16), (1001, 256, 130, 12), (11008, 4096, 4096, 64)])
+def test_backward_without_dx_gives_the_same_lora_gradients(q, n, k, m, r):
+    # a first layer needs no dX: skipping that GEMM (and its stream-K slots in
+    # the workspace) must leave dA and dB bit for bit as in the full backward,
+    # and those match the oracle
+    alpha = 16.0
+    t = _problem(n, k, m, r, seed=5 * n + m)
+    qw = q.qlora_quantize_nf4(t["w"].cuda())
+    x, a, b, dy = (t[k_].cuda() for k_ in ("x", "a", "b", "dy"))
+    _, u = q.qlora_linear_fwd_ex(qw, x, a, b, alpha, path=q.FWD_GEMM)
+    ws = torch.empty(q.qlora_workspace_bytes(m, n, k, r) + 256, dtype=torch.uint8, device="cuda")
+    _, da1, db1 = q.qlora_linear_bwd(qw, x, u, dy, a, b, alpha, ws=ws)
+    none, da2, db2 = q.qlora_linear_bwd(qw, x, u, dy, a, b, alpha, ws=ws, want_dx=False)
+    torch.cuda.synchronize()
+    assert none is None
+    assert torch.equal(da1, da2) and torch.equal(db1, db2)
+    if m <= 512:
+        o = _oracle_quant(t["w"])
+        _, da_ref, db_ref = linear.backward(_np(t["x"]), _np(t["dy"]), _oracle_what(o), _np(t["a"]), _np(t["b"]),
+                                            alpha / r)
+        assert linear.rel_fro(_np(da2), da_ref) <= TOL
+        assert linear.rel_fro(_np(db2), db_ref) <= TOL
+
+
 def test_backward_dx_restores_w_exactly(q):
     # dY = I (tokens = N rows), B = 0: dX[m] = W_hat[m] exactly
     n, k, r = 192, 320, 16
